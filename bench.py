@@ -1,0 +1,447 @@
+"""Benchmark of the Lighthouse layer on B200: one JSON line on stdout (rank 0).
+
+A step is one forward and one backward pass of the layer (pyramid + scores,
+top-K + order, gather, S x S causal attention, scatter-back, and the three
+backward stages) over one batch of synthetic Q, K, V, dO already resident in
+HBM.  Default workload: 98,304 tokens, 16 heads, d = 64, bf16, p = 4, L = 3,
+k = 1536 (S = 18,432).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+replica of the workload (independent (batch, head) problems, no data-path
+collective): weak scaling, value = all ranks' tokens / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_hierarchical_b200.synth import WORKLOADS, make_workload_inputs  # noqa: E402
+
+METRIC = "Lighthouse layer Mtok/s fwd & fwd+bwd at 98K/512K; % HBM/TC roofline"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the layer, stage by stage (the same kernels lh_forward / lh_backward run)
+# ---------------------------------------------------------------------------
+
+STAGES = ("pyramid_score", "topk", "gather", "attn_fwd", "scatter",
+          "scatter_bwd", "attn_bwd", "gather_bwd")
+# kernels each stage launches (lh_topk also issues one cudaMemsetAsync)
+LAUNCHES = {"pyramid_score": 1, "topk": 5, "gather": 1, "attn_fwd": 1, "scatter": 1,
+            "scatter_bwd": 1, "attn_bwd": 2, "gather_bwd": 1}
+
+
+class Layer:
+    """Pre-allocated buffers and stage calls through the C ABI."""
+
+    def __init__(self, lh, w, Q, K, V, dO):
+        import ctypes
+        self.lh, self.w = lh, w
+        self.pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+        self.Q, self.K, self.V, self.dO = Q, K, V, dO
+        dev = Q.device
+        self.ctx = lh.Context(self.pl, dev)
+        self.ws = lh.Workspace(self.pl, dev)
+        self.O = torch.empty_like(Q)
+        self.dQ, self.dK, self.dV = torch.empty_like(Q), torch.empty_like(Q), torch.empty_like(Q)
+        r = self.pl.raw
+        base_c, base_w = self.ctx.buf.data_ptr(), self.ws.buf.data_ptr()
+        P = ctypes.c_void_p
+        self.p = {
+            "sel": P(base_c + r.ctx_sel_idx), "slot": P(base_c + r.ctx_slot_of),
+            "Qg": P(base_c + r.ctx_Qg), "Kg": P(base_c + r.ctx_Kg), "Vg": P(base_c + r.ctx_Vg),
+            "Og": P(base_c + r.ctx_Og), "lse": P(base_c + r.ctx_lse),
+            "pQ": P(base_w + r.ws_pyrQ), "pK": P(base_w + r.ws_pyrK), "pV": P(base_w + r.ws_pyrV),
+            "scores": P(base_w + r.ws_scores), "tws": P(base_w + r.ws_topk),
+            "dOg": P(base_w + r.ws_dOg), "D": P(base_w + r.ws_D), "dQg": P(base_w + r.ws_dQg),
+            "dKg": P(base_w + r.ws_dKg), "dVg": P(base_w + r.ws_dVg), "aws": P(base_w + r.ws_attn),
+        }
+        self.t = {n: P(getattr(self, n).data_ptr()) for n in ("Q", "K", "V", "O", "dO", "dQ", "dK", "dV")}
+
+    def stage(self, name, st):
+        L, pl, p, t, r = self.lh.LIB, self.pl.byref(), self.p, self.t, self.pl.raw
+        BH, S, code = self.pl.BH, self.pl.S, r.c.dtype
+        ck = self.lh._check
+        if name == "pyramid_score":
+            ck(L.lh_pyramid_score(pl, t["Q"], t["K"], t["V"], p["pQ"], p["pK"], p["pV"], p["scores"], st), name)
+        elif name == "topk":
+            ck(L.lh_topk(pl, p["scores"], p["sel"], p["slot"], p["tws"], r.topk_ws_bytes, st), name)
+        elif name == "gather":
+            ck(L.lh_gather(pl, t["Q"], t["K"], t["V"], p["pQ"], p["pK"], p["pV"], p["sel"],
+                           p["Qg"], p["Kg"], p["Vg"], st), name)
+        elif name == "attn_fwd":
+            ck(L.lh_attn_fwd(BH, S, 64, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], st), name)
+        elif name == "scatter":
+            ck(L.lh_scatter(pl, p["Og"], p["slot"], t["O"], st), name)
+        elif name == "scatter_bwd":
+            ck(L.lh_scatter_bwd(pl, t["dO"], p["Og"], p["sel"], p["dOg"], p["D"], st), name)
+        elif name == "attn_bwd":
+            ck(L.lh_attn_bwd(BH, S, 64, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], p["dOg"],
+                             p["D"], p["dQg"], p["dKg"], p["dVg"], p["aws"], r.attn_bwd_ws_bytes, st), name)
+        elif name == "gather_bwd":
+            ck(L.lh_gather_bwd(pl, p["dQg"], p["dKg"], p["dVg"], p["slot"], t["dQ"], t["dK"], t["dV"], st), name)
+
+    def step(self, st, events=None, backward=True):
+        stages = STAGES if backward else STAGES[:5]
+        for i, s in enumerate(stages):
+            self.stage(s, st)
+            if events is not None:
+                events[i].record()
+
+
+def stage_work(pl, w):
+    """Algorithmic bytes (HBM-bound stages) and flops (attention) per step."""
+    r = pl.raw
+    BH, N, S, d, e = pl.BH, w.N, pl.S, w.d, r.elem_bytes
+    row = d * e
+    H = w.B * w.H
+    return {
+        "pyramid_score": ("bytes", 3 * BH * N * row + 3 * BH * pl.Npyr * row + BH * pl.M * 4),
+        "topk": ("bytes", BH * pl.M * 4 + BH * S * 4 + BH * pl.Ntot * 4),
+        "gather": ("bytes", 2 * 3 * BH * S * row + BH * S * 4),
+        "attn_fwd": ("flops", 2 * H * S * (S + 1) * d),
+        "scatter": ("bytes", BH * S * row + BH * pl.Ntot * 4 + BH * N * row),
+        "scatter_bwd": ("bytes", BH * N * row + 2 * BH * S * row + BH * S * 4 * 2),
+        "attn_bwd": ("flops", 5 * H * S * (S + 1) * d),
+        "gather_bwd": ("bytes", 3 * BH * S * row + BH * pl.Ntot * 4 + 3 * BH * N * row),
+    }
+
+
+# ---------------------------------------------------------------------------
+# reference arm / CPU baseline: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+
+def oracle_head_seconds(w, Qh, Kh, Vh, dOh):
+    from oracle import lighthouse as oracle
+    mode = "bf16" if w.dtype == "bf16" else "f32"
+    sz = oracle.sizes(w.N, w.p, w.L, w.k)
+    t0 = time.perf_counter()
+    ctx = oracle.head_forward(Qh, Kh, Vh, sz, mode)
+    oracle.head_backward(ctx, dOh, sz, mode)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_sample_inputs(w, seed, head):
+    """One (b, h) head of the workload's seeded inputs, as fp64 arrays."""
+    Q, K, V, dO = make_workload_inputs(w, seed=seed, device="cpu")
+    pick = lambda x: x[0, head].double().numpy()
+    return pick(Q), pick(K), pick(V), pick(dO)
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    heads = w.B * w.H
+    Qh, Kh, Vh, dOh = cpu_sample_inputs(w, 0, 0)
+    # warm-up on a small slice of the same head (numpy / BLAS start-up)
+    from oracle import lighthouse as oracle
+    small = oracle.sizes(4096, w.p, w.L, min(w.k, 16))
+    mode = "bf16" if w.dtype == "bf16" else "f32"
+    for _ in range(max(0, args.warmup)):
+        c = oracle.head_forward(Qh[:4096], Kh[:4096], Vh[:4096], small, mode)
+        oracle.head_backward(c, dOh[:4096], small, mode)
+    secs = [oracle_head_seconds(w, Qh, Kh, Vh, dOh) for _ in range(args.steps)]
+    per_step = statistics.mean(secs) * heads  # whole layer: all (b, h) heads
+    value = w.B * w.N / per_step / 1e6
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"one (b,h) head of {heads} per step, full forward+backward of "
+                                   f"that head; time x {heads} heads"},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, n):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "p": w.p, "L": w.L,
+            "k": w.k, "global_batch": w.B * n, "seq_len": w.N, "parallelism": f"replicas{n}",
+            "l2": "inputs larger than L2 (Q, K, V, dO 201 MB each at 98K)"}
+
+
+# ---------------------------------------------------------------------------
+# main arm
+# ---------------------------------------------------------------------------
+
+
+def timed_steps(layer, st, steps, backward=True):
+    n = len(STAGES) if backward else 5
+    start = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n)] for _ in range(steps)]
+    start.record()
+    for s in range(steps):
+        layer.step(st, evs[s], backward)
+    torch.cuda.synchronize()
+    total = start.elapsed_time(evs[-1][-1])
+    per_stage = [0.0] * n
+    for s in range(steps):
+        prev = start if s == 0 else evs[s - 1][-1]
+        for i in range(n):
+            per_stage[i] += prev.elapsed_time(evs[s][i])
+            prev = evs[s][i]
+    return total / steps, [x / steps for x in per_stage]
+
+
+def dense_sdpa_ms(H, N, steps=3, backward=True):
+    q = torch.randn(1, H, N, 64, device="cuda", dtype=torch.bfloat16, requires_grad=backward)
+    k = torch.randn_like(q, requires_grad=backward)
+    v = torch.randn_like(q, requires_grad=backward)
+    g = torch.randn_like(q)
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+
+    def once():
+        o = sdpa(q, k, v, is_causal=True)
+        if backward:
+            o.backward(g)
+    once()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        once()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="lighthouse", choices=["lighthouse", "reference"])
+    ap.add_argument("--workload", default="98k_k1536", choices=list(WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true", help="skip comparators and the CPU baseline")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from long_context_hierarchical_b200 import lh
+
+    Q, K, V, dO = make_workload_inputs(w, seed=rank, device="cuda")
+    layer = Layer(lh, w, Q, K, V, dO)
+    st = torch.cuda.current_stream()
+    stp = lh._stream(st)
+    for _ in range(max(3, args.warmup)):
+        layer.step(stp)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ms, per_stage = timed_steps(layer, stp, args.steps)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    lh.device_status()
+
+    tokens = w.B * w.N * world
+    value = tokens / (ms * 1e-3) / 1e6
+    peaks = load_peaks()
+    work = stage_work(layer.pl, w)
+    stages = {}
+    for name, t_ms in zip(STAGES, per_stage):
+        kind, amount = work[name]
+        if kind == "bytes":
+            gbs = amount / (t_ms * 1e-3) / 1e9
+            stages[name] = {"ms": t_ms, "bytes": amount, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]}
+        else:
+            tf = amount / (t_ms * 1e-3) / 1e12
+            stages[name] = {"ms": t_ms, "flops": amount, "TFLOP/s": tf,
+                            "frac_tensor": tf / peaks["bf16_sus"]}
+    dom = max(STAGES, key=lambda s: stages[s]["ms"])
+    d = stages[dom]
+    if "flops" in d:
+        roof = {"kernel": f"lh_{dom}", "bound": "tensor", "achieved": d["TFLOP/s"],
+                "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": d["frac_tensor"],
+                "traffic": None, "peak_source": f"{peaks['src']} bf16 sustained"}
+    else:
+        roof = {"kernel": f"lh_{dom}", "bound": "hbm", "achieved": d["GB/s"], "peak": peaks["hbm"],
+                "unit": "GB/s", "frac": d["frac_hbm"], "traffic": None,
+                "peak_source": f"{peaks['src']} HBM copy"}
+
+    # end to end through the public API: host buffers, copies inside the timed region
+    hQ, hK, hV, hdO = (x.cpu().pin_memory() for x in (Q, K, V, dO))
+    hO, hdQ, hdK, hdV = (torch.empty_like(hQ).pin_memory() for _ in range(4))
+    dQ, dK, dV, O = layer.dQ, layer.dK, layer.dV, layer.O
+    e2e_steps = max(3, args.steps // 2)
+
+    def e2e_once():
+        Q.copy_(hQ, non_blocking=True)
+        K.copy_(hK, non_blocking=True)
+        V.copy_(hV, non_blocking=True)
+        dO.copy_(hdO, non_blocking=True)
+        lh.forward(layer.pl, Q, K, V, O, layer.ctx, layer.ws)
+        lh.backward(layer.pl, dO, layer.ctx, dQ, dK, dV, layer.ws)
+        for h, dvc in ((hO, O), (hdQ, dQ), (hdK, dK), (hdV, dV)):
+            h.copy_(dvc, non_blocking=True)
+    e2e_once()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_once()
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    nbytes = Q.numel() * Q.element_size()
+
+    extras = {}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        fwd_ms, _ = timed_steps(layer, stp, args.steps, backward=False)
+        extras["fwd_mtok_s"] = w.B * w.N / (fwd_ms * 1e-3) / 1e6
+        extras["fwd_ms"] = fwd_ms
+        try:
+            sd_f = dense_sdpa_ms(w.H, w.N, backward=False)
+            sd_fb = dense_sdpa_ms(w.H, w.N, backward=True)
+            extras["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb,
+                                          "speedup_fwd": sd_f / fwd_ms, "speedup_fwd_bwd": sd_fb / ms}
+        except Exception as e:  # comparator only
+            extras["dense_sdpa_torch"] = {"error": str(e)[:200]}
+        torch.cuda.empty_cache()
+        Qh, Kh, Vh, dOh = cpu_sample_inputs(w, 0, 0)
+        secs = oracle_head_seconds(w, Qh, Kh, Vh, dOh)
+        heads = w.B * w.H
+        cpu = {"value": w.B * w.N / (secs * heads) / 1e6, "unit": "Mtok/s", "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": f"one (b,h) head of {heads}: full forward+backward of that head, "
+                         f"{secs:.1f} s, scaled x {heads} heads"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, world),
+            "roofline": roof, "cpu_baseline": cpu,
+            "e2e": {"value": tokens / (e2e_ms * 1e-3) / 1e6, "unit": "Mtok/s",
+                    "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": sum(LAUNCHES.values()) * args.steps,
+            "clocks": clk, "stages": stages, "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

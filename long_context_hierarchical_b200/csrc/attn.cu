@@ -1,0 +1,48 @@
+// Stage-3 attention dispatch: the storage dtype picks the kernel family.
+#include "host.h"
+
+namespace lh {
+
+cudaError_t launch_attn_fwd_f32(int64_t BH, int64_t S, const float* Q, const float* K,
+                                const float* V, float* O, float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_f32(int64_t BH, int64_t S, const float* Q, const float* K,
+                                const float* V, const float* lse, const float* dO,
+                                const float* D, float* dQ, float* dK, float* dV, cudaStream_t st);
+cudaError_t launch_rowdot(int64_t rows, int dtype, const void* dO, const void* O, float* D,
+                          cudaStream_t st);
+cudaError_t launch_attn_fwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
+                                void* O, float* lse, cudaStream_t st);
+cudaError_t launch_attn_bwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
+                                const float* lse, const void* dO, const float* D, void* dQ,
+                                void* dK, void* dV, cudaStream_t st);
+
+int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype) {
+  (void)dtype;
+  return ((BH * S * 4) + 255) & ~int64_t(255);  // D when the caller passes none
+}
+
+cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
+                            const void* Vg, void* Og, float* lse, cudaStream_t st) {
+  if (dtype == LH_F32)
+    return launch_attn_fwd_f32(BH, S, (const float*)Qg, (const float*)Kg, (const float*)Vg,
+                               (float*)Og, lse, st);
+  return launch_attn_fwd_mma(BH, S, Qg, Kg, Vg, Og, lse, st);
+}
+
+cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
+                            const void* Vg, const void* Og, const float* lse, const void* dOg,
+                            const float* D, void* dQg, void* dKg, void* dVg, void* ws,
+                            cudaStream_t st) {
+  if (D == nullptr) {
+    float* Dw = static_cast<float*>(ws);
+    cudaError_t e = launch_rowdot(BH * S, dtype, dOg, Og, Dw, st);
+    if (e != cudaSuccess) return e;
+    D = Dw;
+  }
+  if (dtype == LH_F32)
+    return launch_attn_bwd_f32(BH, S, (const float*)Qg, (const float*)Kg, (const float*)Vg, lse,
+                               (const float*)dOg, D, (float*)dQg, (float*)dKg, (float*)dVg, st);
+  return launch_attn_bwd_mma(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, st);
+}
+
+}  // namespace lh

@@ -1,0 +1,375 @@
+// Stage 2b: joint top-K over the candidate levels and the causal order of the
+// gathered sub-sequence.
+//
+// Selection (skill card "lighthouse-attention", stage 2 "打分与选择";
+// gist.science Technical Summary 2.B): per (batch, head), the Ksel candidates
+// with the largest scores are kept, ties going to the lower level-major flat
+// index, and every coarsest-level entry is kept.  The pages' kernel splits the
+// score stream into 2048-entry chunks with per-CTA register top-128 buffers
+// (skill card, "Kernel Design"); here the selection is an exact radix select
+// on a unique 64-bit key, because only the threshold is needed:
+//
+//   key(f) = orderable(score_f) << 32 | (0xffffffff - f)
+//
+// Larger keys are better and no two are equal, so "f is selected" is exactly
+// key(f) >= kappa where kappa is the Ksel-th largest key.  kappa is found with
+// two 12-bit histogram passes over the score bits, a compaction of the few
+// candidates left in the threshold bucket, and an 8-bit radix select on those.
+//
+// Order (stage 3 "密集子序列注意力"; gist.science 2.C "topologically sorted"):
+// selected entries are laid out by (last token of the span, level), which is
+// a walk over tokens t with, at each t, the levels l whose spans end at t
+// ((t + 1) % p^l == 0).  A count per token block, a scan of the block counts
+// and a rewrite give each selected entry its slot with no sort.
+//
+// Grid-wide phases are separate launches, and the reduction that closes a
+// phase runs in the last block to finish (an atomic ticket); no block ever
+// waits for another.
+#include "host.h"
+
+namespace lh {
+namespace {
+
+constexpr int kHistBins = 4096;
+constexpr int kSelThreads = 512;
+constexpr int kChunk = 8192;       // candidates per block in the histogram passes
+constexpr int kOrdThreads = 256;
+constexpr int kTokPerThread = 8;
+constexpr int kTokBlock = kOrdThreads * kTokPerThread;  // tokens per order block
+
+struct HeadState {
+  uint32_t b1, need1;      // bucket of the top 12 score bits, rank left inside it
+  uint32_t b2, need2;      // bucket of the next 12 bits, rank left inside it
+  uint32_t list_count;     // candidates compacted for the final select
+  uint32_t ticket1, ticket2, ticket3, ticket_count;
+  uint32_t pad[3];
+  unsigned long long kappa;
+  unsigned long long pad2;
+};
+static_assert(sizeof(HeadState) == 64, "HeadState is 64 bytes");
+
+struct Layout {
+  int64_t hist1, hist2, state, blockcnt, list, zero_bytes, total;
+};
+
+int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+Layout layout(const lh_plan& p) {
+  const int64_t BH = (int64_t)p.c.B * p.c.H;
+  const int64_t nblk = (p.c.N + kTokBlock - 1) / kTokBlock;
+  Layout l{};
+  int64_t o = 0;
+  l.hist1 = o; o += BH * kHistBins * 4;
+  l.hist2 = o; o += BH * kHistBins * 4;
+  l.state = o; o += BH * (int64_t)sizeof(HeadState);
+  l.zero_bytes = o;
+  o = align256(o);
+  l.blockcnt = o; o = align256(o + BH * nblk * 4);
+  l.list = o; o = align256(o + BH * p.M * 8);
+  l.total = o;
+  return l;
+}
+
+__device__ __forceinline__ uint32_t orderable(float s) {
+  if (s == 0.f) s = 0.f;  // -0 and +0 are the same score
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long full_key(float s, int64_t f) {
+  return ((unsigned long long)orderable(s) << 32) | (0xffffffffull - (unsigned long long)f);
+}
+
+// Exclusive scan of one value per thread over a block of NT threads.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    constexpr int NW = NT / 32;
+    uint32_t w = lane < NW ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NW) warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const uint32_t before = warp == 0 ? 0 : warp_sums[warp - 1];
+  if (total) *total = warp_sums[NT / 32 - 1];
+  const uint32_t r = before + x - v;
+  __syncthreads();
+  return r;
+}
+
+// Takes a ticket after this block's global writes; true in the last block.
+__device__ __forceinline__ bool last_block(uint32_t* ticket, uint32_t nblocks) {
+  __shared__ bool s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == nblocks - 1;
+  __syncthreads();
+  if (s_last) __threadfence();
+  return s_last;
+}
+
+// In the last block: find the bucket where the rank `need` (1-based, from the
+// top) falls in hist[0..4095]; returns bucket and the rank left inside it.
+__device__ void find_bucket(const uint32_t* hist, uint32_t need, uint32_t* out_b, uint32_t* out_need) {
+  __shared__ uint32_t warp_sums[kSelThreads / 32];
+  constexpr int PER = kHistBins / kSelThreads;  // 8 bins per thread, descending
+  const int t = threadIdx.x;
+  // thread t owns bins [4096 - 8(t+1), 4096 - 8t), i.e. thread 0 the top bins
+  const int hi = kHistBins - PER * t;
+  uint32_t h[PER];
+  uint32_t sum = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    h[i] = __ldcg(hist + hi - 1 - i);
+    sum += h[i];
+  }
+  const uint32_t above = block_excl_scan<kSelThreads>(sum, warp_sums, nullptr);
+  if (above < need && need <= above + sum) {
+    uint32_t cum = above;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      if (cum + h[i] >= need) {
+        *out_b = hi - 1 - i;
+        *out_need = need - cum;
+        break;
+      }
+      cum += h[i];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+hist1_kernel(Geo g, const float* __restrict__ scores, uint32_t* hist1, HeadState* state) {
+  __shared__ uint32_t h[kHistBins];
+  const int64_t bh = blockIdx.y;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) h[i] = 0;
+  __syncthreads();
+  const float* s = scores + bh * g.M;
+  const int64_t f0 = (int64_t)blockIdx.x * kChunk;
+  const int64_t f1 = min(g.M, f0 + kChunk);
+  for (int64_t f = f0 + threadIdx.x; f < f1; f += kSelThreads) atomicAdd(&h[orderable(s[f]) >> 20], 1u);
+  __syncthreads();
+  uint32_t* gh = hist1 + bh * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads)
+    if (h[i]) atomicAdd(gh + i, h[i]);
+  if (last_block(&state[bh].ticket1, gridDim.x))
+    find_bucket(gh, (uint32_t)g.Ksel, &state[bh].b1, &state[bh].need1);
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+hist2_kernel(Geo g, const float* __restrict__ scores, uint32_t* hist2, HeadState* state) {
+  __shared__ uint32_t h[kHistBins];
+  const int64_t bh = blockIdx.y;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) h[i] = 0;
+  __syncthreads();
+  const uint32_t b1 = __ldcg(&state[bh].b1);
+  const float* s = scores + bh * g.M;
+  const int64_t f0 = (int64_t)blockIdx.x * kChunk;
+  const int64_t f1 = min(g.M, f0 + kChunk);
+  for (int64_t f = f0 + threadIdx.x; f < f1; f += kSelThreads) {
+    const uint32_t k = orderable(s[f]);
+    if ((k >> 20) == b1) atomicAdd(&h[(k >> 8) & 0xfffu], 1u);
+  }
+  __syncthreads();
+  uint32_t* gh = hist2 + bh * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += kSelThreads)
+    if (h[i]) atomicAdd(gh + i, h[i]);
+  if (last_block(&state[bh].ticket2, gridDim.x))
+    find_bucket(gh, __ldcg(&state[bh].need1), &state[bh].b2, &state[bh].need2);
+}
+
+// Compacts the candidates of the threshold bucket (top 24 key bits fixed);
+// the last block then resolves the remaining 8 score bits and the index by a
+// radix select over 5 digits of 8 bits.
+__global__ void __launch_bounds__(kSelThreads)
+collect_kernel(Geo g, const float* __restrict__ scores, unsigned long long* list, HeadState* state) {
+  const int64_t bh = blockIdx.y;
+  HeadState* st = &state[bh];
+  const uint32_t prefix = (__ldcg(&st->b1) << 12) | __ldcg(&st->b2);
+  const float* s = scores + bh * g.M;
+  unsigned long long* lst = list + bh * g.M;
+  const int64_t f0 = (int64_t)blockIdx.x * kChunk;
+  const int64_t f1 = min(g.M, f0 + kChunk);
+  const int lane = threadIdx.x & 31;
+  for (int64_t base = f0; base < f1; base += kSelThreads) {
+    const int64_t f = base + threadIdx.x;
+    bool hit = false;
+    unsigned long long key = 0;
+    if (f < f1) {
+      key = full_key(s[f], f);
+      hit = (uint32_t)(key >> 40) == prefix;
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, hit);
+    if (m) {
+      uint32_t pos = 0;
+      if (lane == 0) pos = atomicAdd(&st->list_count, (uint32_t)__popc(m));
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      if (hit) lst[pos + __popc(m & ((1u << lane) - 1))] = key;
+    }
+  }
+  if (!last_block(&st->ticket3, gridDim.x)) return;
+
+  __shared__ uint32_t h[256];
+  __shared__ uint32_t s_digit, s_need;
+  __shared__ uint32_t warp_sums[kSelThreads / 32];
+  const uint32_t cnt = __ldcg(&st->list_count);
+  uint32_t need = __ldcg(&st->need2);
+  unsigned long long rem = 0;        // resolved low 40 bits so far
+  unsigned long long rem_mask = 0;   // which of them are resolved
+  for (int shift = 32; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) h[i] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < cnt; i += kSelThreads) {
+      const unsigned long long k = __ldcg(lst + i) & 0xffffffffffull;
+      if ((k & rem_mask) == rem) atomicAdd(&h[(k >> shift) & 0xffu], 1u);
+    }
+    __syncthreads();
+    // descending scan over 256 bins: thread t < 256 takes bin 255 - t
+    const int t = threadIdx.x;
+    const uint32_t v = t < 256 ? h[255 - t] : 0;
+    const uint32_t above = block_excl_scan<kSelThreads>(v, warp_sums, nullptr);
+    if (t < 256 && above < need && need <= above + v) {
+      s_digit = 255 - t;
+      s_need = need - above;
+    }
+    __syncthreads();
+    rem |= (unsigned long long)s_digit << shift;
+    rem_mask |= 0xffull << shift;
+    need = s_need;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) st->kappa = ((unsigned long long)prefix << 40) | rem;
+}
+
+// --- ordering -------------------------------------------------------------
+
+struct SelCtx {
+  const float* s;  // this head's candidate scores
+  unsigned long long kappa;
+  bool any;        // Ksel > 0
+};
+
+__device__ __forceinline__ bool is_selected(const Geo& g, const SelCtx& c, int l, int64_t i) {
+  if (l == g.L - 1) return true;
+  if (!c.any) return false;
+  const int64_t f = g.flat_off[l] + i;
+  return full_key(c.s[f], f) >= c.kappa;
+}
+
+// Number of selected entries whose span ends at tokens [t0, t1).
+__device__ __forceinline__ uint32_t count_range(const Geo& g, const SelCtx& c, int64_t t0, int64_t t1) {
+  uint32_t n = 0;
+  for (int64_t t = t0; t < t1; ++t) {
+    for (int l = 0; l < g.L; ++l) {
+      const int sh = g.logp * l;  // p^l = 2^sh
+      if (((t + 1) & ((int64_t(1) << sh) - 1)) != 0) break;  // coarser levels fail too
+      n += is_selected(g, c, l, ((t + 1) >> sh) - 1);
+    }
+  }
+  return n;
+}
+
+__global__ void __launch_bounds__(kOrdThreads)
+order_count_kernel(Geo g, const float* __restrict__ scores, const HeadState* state,
+                   uint32_t* blockcnt, HeadState* wstate, int64_t nblk) {
+  __shared__ uint32_t warp_sums[kOrdThreads / 32];
+  const int64_t bh = blockIdx.y;
+  SelCtx c{scores + bh * g.M, state[bh].kappa, g.Ksel > 0};
+  const int64_t t0 = (int64_t)blockIdx.x * kTokBlock + threadIdx.x * kTokPerThread;
+  const int64_t t1 = min(g.N, t0 + kTokPerThread);
+  const uint32_t mine = t0 < g.N ? count_range(g, c, t0, t1) : 0;
+  uint32_t total;
+  block_excl_scan<kOrdThreads>(mine, warp_sums, &total);
+  uint32_t* bc = blockcnt + bh * nblk;
+  if (threadIdx.x == 0) bc[blockIdx.x] = total;
+  if (!last_block(&wstate[bh].ticket_count, gridDim.x)) return;
+  // Exclusive scan of the block counts, in place.
+  uint32_t carry = 0;
+  for (int64_t base = 0; base < nblk; base += kOrdThreads) {
+    const int64_t i = base + threadIdx.x;
+    const uint32_t v = i < nblk ? __ldcg(bc + i) : 0;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan<kOrdThreads>(v, warp_sums, &tot);
+    if (i < nblk) bc[i] = carry + ex;
+    carry += tot;
+  }
+}
+
+__global__ void __launch_bounds__(kOrdThreads)
+order_write_kernel(Geo g, const float* __restrict__ scores, const HeadState* state,
+                   const uint32_t* blockoff, int32_t* __restrict__ sel_idx,
+                   int32_t* __restrict__ slot_of, int64_t nblk) {
+  __shared__ uint32_t warp_sums[kOrdThreads / 32];
+  const int64_t bh = blockIdx.y;
+  SelCtx c{scores + bh * g.M, state[bh].kappa, g.Ksel > 0};
+  const int64_t t0 = (int64_t)blockIdx.x * kTokBlock + threadIdx.x * kTokPerThread;
+  const int64_t t1 = min(g.N, t0 + kTokPerThread);
+  const uint32_t mine = t0 < g.N ? count_range(g, c, t0, t1) : 0;
+  uint32_t slot = blockoff[bh * nblk + blockIdx.x] +
+                  block_excl_scan<kOrdThreads>(mine, warp_sums, nullptr);
+  int32_t* sel = sel_idx + bh * g.S;
+  int32_t* inv = slot_of + bh * g.Ntot;
+  for (int64_t t = t0; t < t1; ++t) {
+    for (int l = 0; l < g.L; ++l) {
+      const int sh = g.logp * l;
+      if (((t + 1) & ((int64_t(1) << sh) - 1)) != 0) break;
+      const int64_t i = ((t + 1) >> sh) - 1;
+      const int64_t f = g.flat_off[l] + i;
+      if (is_selected(g, c, l, i)) {
+        // slot < S holds whenever exactly Ksel candidates pass; the guard
+        // keeps a wrong threshold from writing past the buffer.
+        if (slot < g.S) sel[slot] = (int32_t)f;
+        inv[f] = slot < g.S ? (int32_t)slot : -1;
+        ++slot;
+      } else {
+        inv[f] = -1;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+int64_t topk_ws_bytes(const lh_plan& plan) { return layout(plan).total; }
+
+cudaError_t launch_topk(const lh_plan& plan, const float* scores, int32_t* sel_idx,
+                        int32_t* slot_of, void* ws, cudaStream_t st) {
+  const Geo g = make_geo(plan);
+  const Layout lay = layout(plan);
+  char* w = static_cast<char*>(ws);
+  uint32_t* hist1 = reinterpret_cast<uint32_t*>(w + lay.hist1);
+  uint32_t* hist2 = reinterpret_cast<uint32_t*>(w + lay.hist2);
+  HeadState* state = reinterpret_cast<HeadState*>(w + lay.state);
+  uint32_t* blockcnt = reinterpret_cast<uint32_t*>(w + lay.blockcnt);
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(w + lay.list);
+  const int64_t nblk = (g.N + kTokBlock - 1) / kTokBlock;
+
+  cudaError_t e = cudaMemsetAsync(w, 0, lay.zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  if (g.Ksel > 0) {
+    const dim3 grid((unsigned)((g.M + kChunk - 1) / kChunk), (unsigned)g.BH);
+    hist1_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, hist1, state);
+    hist2_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, hist2, state);
+    collect_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, list, state);
+  }
+  const dim3 ogrid((unsigned)nblk, (unsigned)g.BH);
+  order_count_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, state, blockcnt, state, nblk);
+  order_write_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, state, blockcnt, sel_idx, slot_of,
+                                                    nblk);
+  return cudaGetLastError();
+}
+
+}  // namespace lh

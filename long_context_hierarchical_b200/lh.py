@@ -1,0 +1,346 @@
+"""Python binding of the Lighthouse C ABI (include/lh.h).
+
+Argument marshalling only: every stage runs in liblh.so's CUDA kernels.
+PyTorch provides device memory and the current stream.  Importing this module
+loads liblh.so and fails loudly if it is missing; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblh.so")
+
+LH_OK, LH_ERR_INVALID_ARG, LH_ERR_UNSUPPORTED, LH_ERR_WORKSPACE, LH_ERR_CUDA, LH_ERR_TIMEOUT = range(6)
+LH_F32, LH_BF16 = 0, 1
+MAX_LEVELS = 8
+DTYPES = {"f32": LH_F32, "bf16": LH_BF16}
+TORCH_DTYPE = {LH_F32: torch.float32, LH_BF16: torch.bfloat16}
+
+# Every exported name declared in include/lh.h.
+EXPORTS = (
+    "lh_plan_init", "lh_pyramid", "lh_score", "lh_pyramid_score", "lh_topk", "lh_gather",
+    "lh_attn_fwd", "lh_attn_bwd_ws_bytes", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd",
+    "lh_gather_bwd", "lh_forward", "lh_backward", "lh_device_status", "lh_status_string",
+    "lh_last_error", "lh_plan_bytes",
+)
+
+
+class LhConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "p", "L", "k", "dtype")]
+
+
+_I64 = ctypes.c_int64
+
+
+class LhPlan(ctypes.Structure):
+    _fields_ = [
+        ("c", LhConfig),
+        ("P", _I64 * MAX_LEVELS),
+        ("n", _I64 * MAX_LEVELS),
+        ("flat_off", _I64 * (MAX_LEVELS + 1)),
+        ("pyr_off", _I64 * MAX_LEVELS),
+    ] + [(n, _I64) for n in (
+        "Ntot", "Npyr", "M", "Ksel", "S", "elem_bytes",
+        "ctx_bytes", "ws_bytes", "topk_ws_bytes", "attn_bwd_ws_bytes",
+        "ctx_sel_idx", "ctx_slot_of", "ctx_Qg", "ctx_Kg", "ctx_Vg", "ctx_Og", "ctx_lse",
+        "ws_pyrQ", "ws_pyrK", "ws_pyrV", "ws_scores", "ws_topk",
+        "ws_dOg", "ws_D", "ws_dQg", "ws_dKg", "ws_dVg", "ws_attn")]
+
+
+class LighthouseError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({detail})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m long_context_hierarchical_b200.build`"
+            " (the Lighthouse layer has no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    PLAN = ctypes.POINTER(LhPlan)
+    sig = {
+        "lh_plan_init": (ctypes.POINTER(LhConfig), PLAN),
+        "lh_pyramid": (PLAN, P, P, P, P, P, P, P),
+        "lh_score": (PLAN, P, P, P, P),
+        "lh_pyramid_score": (PLAN, P, P, P, P, P, P, P, P),
+        "lh_topk": (PLAN, P, P, P, P, SZ, P),
+        "lh_gather": (PLAN, P, P, P, P, P, P, P, P, P, P, P),
+        "lh_attn_fwd": (I64, I64, I32, I32, P, P, P, P, P, P),
+        "lh_attn_bwd": (I64, I64, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P),
+        "lh_scatter": (PLAN, P, P, P, P),
+        "lh_scatter_bwd": (PLAN, P, P, P, P, P, P),
+        "lh_gather_bwd": (PLAN, P, P, P, P, P, P, P, P),
+        "lh_forward": (PLAN, P, P, P, P, P, P, P),
+        "lh_backward": (PLAN, P, P, P, P, P, P, P),
+        "lh_device_status": (ctypes.c_int,),
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = list(args)
+        f.restype = ctypes.c_int
+    lib.lh_attn_bwd_ws_bytes.argtypes = [I64, I64, I32, I32]
+    lib.lh_attn_bwd_ws_bytes.restype = I64
+    lib.lh_status_string.argtypes = [ctypes.c_int]
+    lib.lh_status_string.restype = ctypes.c_char_p
+    lib.lh_last_error.argtypes = []
+    lib.lh_last_error.restype = ctypes.c_char_p
+    lib.lh_plan_bytes.argtypes = []
+    lib.lh_plan_bytes.restype = I64
+    if lib.lh_plan_bytes() != ctypes.sizeof(LhPlan):
+        raise ImportError("lh_plan layout of liblh.so does not match this binding")
+    return lib
+
+
+LIB = _load()
+
+
+def _check(status: int, where: str):
+    if status != LH_OK:
+        detail = (LIB.lh_last_error() or b"").decode() or LIB.lh_status_string(status).decode()
+        raise LighthouseError(status, where, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class Plan:
+    """Sizes and buffer layout of one layer configuration (from lh_plan_init)."""
+    raw: LhPlan
+
+    @property
+    def S(self):
+        return self.raw.S
+
+    @property
+    def M(self):
+        return self.raw.M
+
+    @property
+    def Ntot(self):
+        return self.raw.Ntot
+
+    @property
+    def Npyr(self):
+        return self.raw.Npyr
+
+    @property
+    def Ksel(self):
+        return self.raw.Ksel
+
+    @property
+    def BH(self):
+        return self.raw.c.B * self.raw.c.H
+
+    @property
+    def dtype(self):
+        return TORCH_DTYPE[self.raw.c.dtype]
+
+    def byref(self):
+        return ctypes.byref(self.raw)
+
+
+def plan(B: int, H: int, N: int, d: int = 64, p: int = 4, L: int = 3, k: int = 0,
+         dtype: str = "bf16") -> Plan:
+    cfg = LhConfig(B, H, N, d, p, L, k, DTYPES[dtype])
+    raw = LhPlan()
+    _check(LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(raw)), "lh_plan_init")
+    return Plan(raw)
+
+
+def _empty(shape, dtype, device):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def _bytes(n, device):
+    return torch.empty(max(int(n), 16), dtype=torch.uint8, device=device)
+
+
+# --- stages -----------------------------------------------------------------
+
+
+def pyramid_score(pl: Plan, Q, K, V, stream=None):
+    """Levels 1..L-1 of Q, K, V ([B,H,Npyr,d] each) and candidate scores [B,H,M]."""
+    c = pl.raw.c
+    dev = Q.device
+    pyr = [_empty((c.B, c.H, max(pl.Npyr, 1), c.d), Q.dtype, dev) for _ in range(3)]
+    scores = _empty((c.B, c.H, max(pl.M, 1)), torch.float32, dev)
+    _check(LIB.lh_pyramid_score(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), *map(_ptr, pyr),
+                                _ptr(scores), _stream(stream)), "lh_pyramid_score")
+    return pyr, scores
+
+
+def pyramid(pl: Plan, Q, K, V, stream=None):
+    c = pl.raw.c
+    pyr = [_empty((c.B, c.H, max(pl.Npyr, 1), c.d), Q.dtype, Q.device) for _ in range(3)]
+    _check(LIB.lh_pyramid(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), *map(_ptr, pyr),
+                          _stream(stream)), "lh_pyramid")
+    return pyr
+
+
+def score(pl: Plan, Q, K, stream=None):
+    c = pl.raw.c
+    scores = _empty((c.B, c.H, max(pl.M, 1)), torch.float32, Q.device)
+    _check(LIB.lh_score(pl.byref(), _ptr(Q), _ptr(K), _ptr(scores), _stream(stream)), "lh_score")
+    return scores
+
+
+def topk(pl: Plan, scores, stream=None):
+    """(sel_idx [B,H,S] int32, slot_of [B,H,Ntot] int32) from scores [B,H,M]."""
+    c = pl.raw.c
+    dev = scores.device
+    sel = _empty((c.B, c.H, pl.S), torch.int32, dev)
+    inv = _empty((c.B, c.H, pl.Ntot), torch.int32, dev)
+    ws = _bytes(pl.raw.topk_ws_bytes, dev)
+    _check(LIB.lh_topk(pl.byref(), _ptr(scores), _ptr(sel), _ptr(inv), _ptr(ws), ws.numel(),
+                       _stream(stream)), "lh_topk")
+    return sel, inv
+
+
+def gather(pl: Plan, Q, K, V, pyr, sel_idx, stream=None):
+    c = pl.raw.c
+    out = [_empty((c.B, c.H, pl.S, c.d), Q.dtype, Q.device) for _ in range(3)]
+    _check(LIB.lh_gather(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), *map(_ptr, pyr), _ptr(sel_idx),
+                         *map(_ptr, out), _stream(stream)), "lh_gather")
+    return out
+
+
+def _dtype_code(t):
+    return LH_BF16 if t.dtype == torch.bfloat16 else LH_F32
+
+
+def attn_fwd(Qg, Kg, Vg, stream=None):
+    """Causal attention on [..., S, d] tensors: (O, lse[..., S] natural log)."""
+    S, d = Qg.shape[-2], Qg.shape[-1]
+    BH = Qg.numel() // (S * d)
+    O = torch.empty_like(Qg)
+    lse = _empty(Qg.shape[:-1], torch.float32, Qg.device)
+    _check(LIB.lh_attn_fwd(BH, S, d, _dtype_code(Qg), _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(O),
+                           _ptr(lse), _stream(stream)), "lh_attn_fwd")
+    return O, lse
+
+
+def attn_bwd(Qg, Kg, Vg, Og, lse, dOg, D=None, stream=None):
+    S, d = Qg.shape[-2], Qg.shape[-1]
+    BH = Qg.numel() // (S * d)
+    code = _dtype_code(Qg)
+    dQ, dK, dV = torch.empty_like(Qg), torch.empty_like(Kg), torch.empty_like(Vg)
+    ws = _bytes(LIB.lh_attn_bwd_ws_bytes(BH, S, d, code), Qg.device)
+    _check(LIB.lh_attn_bwd(BH, S, d, code, _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(Og), _ptr(lse),
+                           _ptr(dOg), _ptr(D), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws), ws.numel(),
+                           _stream(stream)), "lh_attn_bwd")
+    return dQ, dK, dV
+
+
+def scatter(pl: Plan, Og, slot_of, stream=None):
+    c = pl.raw.c
+    O = _empty((c.B, c.H, c.N, c.d), Og.dtype, Og.device)
+    _check(LIB.lh_scatter(pl.byref(), _ptr(Og), _ptr(slot_of), _ptr(O), _stream(stream)),
+           "lh_scatter")
+    return O
+
+
+def scatter_bwd(pl: Plan, dO, Og, sel_idx, stream=None):
+    c = pl.raw.c
+    dOg = _empty((c.B, c.H, pl.S, c.d), dO.dtype, dO.device)
+    D = _empty((c.B, c.H, pl.S), torch.float32, dO.device)
+    _check(LIB.lh_scatter_bwd(pl.byref(), _ptr(dO), _ptr(Og), _ptr(sel_idx), _ptr(dOg), _ptr(D),
+                              _stream(stream)), "lh_scatter_bwd")
+    return dOg, D
+
+
+def gather_bwd(pl: Plan, dQg, dKg, dVg, slot_of, stream=None):
+    c = pl.raw.c
+    out = [_empty((c.B, c.H, c.N, c.d), dQg.dtype, dQg.device) for _ in range(3)]
+    _check(LIB.lh_gather_bwd(pl.byref(), _ptr(dQg), _ptr(dKg), _ptr(dVg), _ptr(slot_of),
+                             *map(_ptr, out), _stream(stream)), "lh_gather_bwd")
+    return out
+
+
+# --- whole layer --------------------------------------------------------------
+
+
+class Context:
+    """The forward-to-backward buffer of one lh_forward call, with typed views."""
+
+    def __init__(self, pl: Plan, device):
+        self.plan = pl
+        self.buf = _bytes(pl.raw.ctx_bytes, device)
+
+    def _view(self, off, shape, dtype):
+        n = 1
+        for s in shape:
+            n *= s
+        nbytes = n * torch.tensor([], dtype=dtype).element_size()
+        return self.buf[off: off + nbytes].view(dtype).view(shape)
+
+    @property
+    def sel_idx(self):
+        c = self.plan.raw.c
+        return self._view(self.plan.raw.ctx_sel_idx, (c.B, c.H, self.plan.S), torch.int32)
+
+    @property
+    def slot_of(self):
+        c = self.plan.raw.c
+        return self._view(self.plan.raw.ctx_slot_of, (c.B, c.H, self.plan.Ntot), torch.int32)
+
+    def gathered(self, name):
+        c = self.plan.raw.c
+        off = getattr(self.plan.raw, "ctx_" + name)
+        return self._view(off, (c.B, c.H, self.plan.S, c.d), self.plan.dtype)
+
+    @property
+    def lse(self):
+        c = self.plan.raw.c
+        return self._view(self.plan.raw.ctx_lse, (c.B, c.H, self.plan.S), torch.float32)
+
+
+class Workspace:
+    def __init__(self, pl: Plan, device):
+        self.buf = _bytes(pl.raw.ws_bytes, device)
+
+
+def forward(pl: Plan, Q, K, V, O=None, ctx: Context | None = None, ws: Workspace | None = None,
+            stream=None):
+    """O = Lighthouse(Q, K, V); returns (O, ctx)."""
+    dev = Q.device
+    if O is None:
+        O = torch.empty_like(Q)
+    if ctx is None:
+        ctx = Context(pl, dev)
+    if ws is None:
+        ws = Workspace(pl, dev)
+    _check(LIB.lh_forward(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(ctx.buf),
+                          _ptr(ws.buf), _stream(stream)), "lh_forward")
+    return O, ctx
+
+
+def backward(pl: Plan, dO, ctx: Context, dQ=None, dK=None, dV=None, ws: Workspace | None = None,
+             stream=None):
+    """(dQ, dK, dV) from dO and the ctx of the matching forward."""
+    if dQ is None:
+        dQ, dK, dV = torch.empty_like(dO), torch.empty_like(dO), torch.empty_like(dO)
+    if ws is None:
+        ws = Workspace(pl, dO.device)
+    _check(LIB.lh_backward(pl.byref(), _ptr(dO), _ptr(ctx.buf), _ptr(dQ), _ptr(dK), _ptr(dV),
+                           _ptr(ws.buf), _stream(stream)), "lh_backward")
+    return dQ, dK, dV
+
+
+def device_status(reset: bool = True):
+    _check(LIB.lh_device_status(1 if reset else 0), "lh_device_status")

@@ -1,0 +1,103 @@
+"""The C-ABI library on the host: exports, plan validation, argument checks.
+
+Nothing here launches a kernel, so these run without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from oracle import lighthouse as oracle
+from long_context_hierarchical_b200 import lh
+from long_context_hierarchical_b200.synth import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "lh.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lh_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_function_is_exported():
+    names = declared_functions()
+    assert len(names) >= 18
+    lib = ctypes.CDLL(lh.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(lh.EXPORTS)
+
+
+def test_plan_struct_matches_binding():
+    assert lh.LIB.lh_plan_bytes() == ctypes.sizeof(lh.LhPlan)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_plan_sizes_match_oracle(name):
+    w = WORKLOADS[name]
+    p = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+    sz = oracle.sizes(w.N, w.p, w.L, w.k)
+    assert (p.S, p.M, p.Ntot, p.Ksel) == (sz.S, sz.M, sz.Ntot, sz.Ksel)
+    assert list(p.raw.flat_off)[: w.L + 1] == sz.flat_off
+    assert p.Npyr == sz.Ntot - w.N
+    assert p.raw.ctx_bytes > 0 and p.raw.ws_bytes > 0
+    for off in ("ctx_sel_idx", "ctx_slot_of", "ctx_Qg", "ctx_Kg", "ctx_Vg", "ctx_Og", "ctx_lse",
+                "ws_pyrQ", "ws_scores", "ws_topk", "ws_dOg", "ws_D", "ws_attn"):
+        assert getattr(p.raw, off) % 256 == 0
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 2, 1000, 64, 4, 3, 1, "bf16"), lh.LH_ERR_INVALID_ARG),   # N % p^(L-1)
+    ((1, 2, 1024, 64, 4, 3, 200, "bf16"), lh.LH_ERR_INVALID_ARG),  # budget > M
+    ((1, 2, 1024, 64, 1, 3, 1, "bf16"), lh.LH_ERR_INVALID_ARG),    # p < 2
+    ((1, 2, 1024, 64, 4, 0, 1, "bf16"), lh.LH_ERR_INVALID_ARG),    # L < 1
+    ((0, 2, 1024, 64, 4, 3, 1, "bf16"), lh.LH_ERR_INVALID_ARG),    # B < 1
+    ((1, 2, 1024, 64, 4, 3, -1, "bf16"), lh.LH_ERR_INVALID_ARG),   # k < 0
+    ((1, 2, 1024, 128, 4, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),   # d = 128
+    ((1, 2, 1152, 64, 3, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # p = 3
+    ((1, 2, 4096, 64, 2, 6, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # L = 6
+    ((1, 2, 4096, 64, 4, 5, 1, "bf16"), None),                     # p^(L-1) = 256: built
+])
+def test_plan_validation(args, status):
+    if status is None:
+        lh.plan(*args)
+        return
+    with pytest.raises(lh.LighthouseError) as e:
+        lh.plan(*args)
+    assert e.value.status == status
+
+
+def test_plan_rejects_unknown_dtype():
+    cfg = lh.LhConfig(1, 2, 1024, 64, 4, 3, 1, 7)
+    out = lh.LhPlan()
+    assert lh.LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(out)) == lh.LH_ERR_UNSUPPORTED
+    assert lh.LIB.lh_plan_init(None, ctypes.byref(out)) == lh.LH_ERR_INVALID_ARG
+
+
+def test_entry_points_reject_bad_pointers_before_launching():
+    p = lh.plan(1, 2, 1024, 64, 4, 3, 8, "bf16")
+    ref = p.byref()
+    good = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced here
+    odd = ctypes.c_void_p((1 << 20) + 8)  # not 16-byte aligned
+    L = lh.LIB
+    assert L.lh_forward(ref, None, good, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
+    assert L.lh_forward(ref, good, good, good, good, good, odd, None) == lh.LH_ERR_INVALID_ARG
+    assert b"aligned" in L.lh_last_error()
+    assert L.lh_backward(ref, good, None, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
+    assert L.lh_topk(ref, good, good, good, good, 16, None) == lh.LH_ERR_WORKSPACE
+    assert L.lh_attn_fwd(2, 100, 128, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_UNSUPPORTED
+    assert L.lh_attn_fwd(0, 100, 64, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
+    assert L.lh_attn_bwd_ws_bytes(2, 100, 64, lh.LH_BF16) >= 2 * 100 * 4
+    assert L.lh_attn_bwd(2, 100, 64, lh.LH_BF16, good, good, good, good, good, good, None, good,
+                         good, good, good, 0, None) == lh.LH_ERR_WORKSPACE
+    # a plan that was not produced by lh_plan_init is refused
+    bad = lh.LhPlan.from_buffer_copy(p.raw)
+    bad.S += 1
+    assert L.lh_scatter(ctypes.byref(bad), good, good, good, None) == lh.LH_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for s in range(6):
+        assert lh.LIB.lh_status_string(s)

@@ -1,0 +1,208 @@
+"""Per-stage and whole-layer parity of the CUDA path against the oracle.
+
+Each stage is fed the oracle's own inputs for that stage (seeded inputs,
+never values from the CUDA path) and compared element by element:
+selection and order bit-exact, scores within 1e-6 relative, pyramid means
+within one rounding step, outputs and gradients within 2e-2 (bf16) or 1e-4
+(fp32) of max(1, |oracle|).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import lighthouse as oracle
+from long_context_hierarchical_b200.synth import make_inputs, make_scores
+from tests.helpers import (TOL, assert_close, assert_pyr_close, np64, oracle_layer, stack)
+
+pytestmark = pytest.mark.gpu
+
+# name: (B, H, N, dtype, p, L, k)
+CASES = {
+    "tiny_f32": (1, 2, 1024, "f32", 4, 3, 32),          # S = 320
+    "8k_bf16": (1, 8, 8192, "bf16", 4, 4, 256),         # S = 3200
+    "p2_ragged": (2, 3, 96, "bf16", 2, 3, 5),           # S = 44: partial tiles
+    "L2": (1, 2, 512, "bf16", 4, 2, 16),                # S = 192
+    "L5": (1, 2, 2048, "bf16", 4, 5, 8),                # p^(L-1) = 256, S = 136
+    "L1_dense": (1, 2, 256, "bf16", 4, 1, 0),           # selection off: S = N
+    "k0": (1, 2, 1024, "bf16", 4, 3, 0),                # coarsest level only: S = 64
+    "kmax": (1, 2, 64, "bf16", 2, 2, 32),               # every candidate: S = 96
+    "f32_p2_L5": (1, 1, 256, "f32", 2, 5, 3),           # S = 40
+    "p2_L4_odd": (1, 2, 200, "bf16", 2, 4, 7),          # N = 25 * 8, S = 67
+}
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module", params=list(CASES))
+def case(request):
+    from long_context_hierarchical_b200 import lh
+    B, H, N, dtype, p, L, k = CASES[request.param]
+    Q, K, V, dO = make_inputs(B, H, N, 64, dtype, seed=0)
+    O, ctxs, sz, grads = oracle_layer(Q, K, V, dO, p, L, k, DT[dtype])
+    pl = lh.plan(B, H, N, 64, p, L, k, dtype)
+    dev = torch.device("cuda")
+    return dict(name=request.param, B=B, H=H, N=N, dt=DT[dtype], p=p, L=L, k=k, lh=lh, pl=pl,
+                Q=Q.to(dev), K=K.to(dev), V=V.to(dev), dO=dO.to(dev), O=O, ctxs=ctxs, sz=sz,
+                grads=grads)
+
+
+def _t(a, dtype, dev="cuda"):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dtype)
+
+
+def _oracle_pyr(c, which):
+    """Levels 1..L-1 of tensor `which` (0,1,2) as one [B,H,Npyr,d] array."""
+    rows = []
+    for row in c["ctxs"]:
+        hs = []
+        for ctx in row:
+            lv = ctx["levels"][which]
+            hs.append(np.concatenate(lv[1:], axis=0) if len(lv) > 1 else np.zeros((1, 64)))
+        rows.append(np.stack(hs))
+    return np.stack(rows)
+
+
+def test_pyramid_and_scores(case):
+    c = case
+    lh, pl = c["lh"], c["pl"]
+    pyr, scores = lh.pyramid_score(pl, c["Q"], c["K"], c["V"])
+    torch.cuda.synchronize()
+    if pl.Npyr > 0:
+        for w in range(3):
+            assert_pyr_close(np64(pyr[w]), _oracle_pyr(c, w), c["dt"], f"pyramid[{w}]")
+    if pl.M > 0:
+        got = np64(scores)
+        exp = stack(c["ctxs"], "cand")
+        rel = np.abs(got - exp) / np.maximum(np.abs(exp), 1e-30)
+        assert rel.max() <= 1e-6, rel.max()
+        # the separate entry points give the fused kernel's bytes
+        assert torch.equal(lh.score(pl, c["Q"], c["K"]), scores)
+    if pl.Npyr > 0:
+        sep = lh.pyramid(pl, c["Q"], c["K"], c["V"])
+        for w in range(3):
+            assert torch.equal(sep[w], pyr[w])
+
+
+def test_topk_on_oracle_scores(case):
+    c = case
+    lh, pl = c["lh"], c["pl"]
+    cand = stack(c["ctxs"], "cand") if pl.M > 0 else np.zeros((c["B"], c["H"], 1))
+    sel, inv = lh.topk(pl, _t(cand, torch.float32))
+    assert np.array_equal(sel.cpu().numpy(), stack(c["ctxs"], "sel_idx"))
+    assert np.array_equal(inv.cpu().numpy(), stack(c["ctxs"], "slot_of"))
+
+
+@pytest.mark.parametrize("distinct", [None, 3, 1])
+def test_topk_ties_and_random_scores(distinct):
+    """Selection on seeded score arrays, including exact ties everywhere."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k = 1, 3, 4096, 4, 4, 40
+    sz = oracle.sizes(N, p, L, k)
+    scores = make_scores(B, H, sz.M, seed=5, distinct=distinct)
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16")
+    sel, inv = lh.topk(pl, scores.cuda())
+    for h in range(H):
+        mask = oracle.select(scores[0, h].double().numpy(), sz)
+        es, ei = oracle.order_selection(mask, sz)
+        assert np.array_equal(sel[0, h].cpu().numpy(), es)
+        assert np.array_equal(inv[0, h].cpu().numpy(), ei)
+
+
+def test_gather(case):
+    c = case
+    lh, pl, dt = c["lh"], c["pl"], c["dt"]
+    pyr = [_t(_oracle_pyr(c, w), dt) for w in range(3)]
+    sel = _t(stack(c["ctxs"], "sel_idx"), torch.int32)
+    out = lh.gather(pl, c["Q"], c["K"], c["V"], pyr, sel)
+    for w, key in enumerate(("Qg", "Kg", "Vg")):
+        assert np.array_equal(np64(out[w]), stack(c["ctxs"], key)), key
+
+
+def test_attention_forward(case):
+    c = case
+    lh, dt = c["lh"], c["dt"]
+    Qg, Kg, Vg = (_t(stack(c["ctxs"], k), dt) for k in ("Qg", "Kg", "Vg"))
+    Og, lse = lh.attn_fwd(Qg, Kg, Vg)
+    assert_close(np64(Og), stack(c["ctxs"], "Og"), dt, "Og")
+    lt = 1e-3 if dt == torch.bfloat16 else 1e-5
+    assert np.max(np.abs(np64(lse) - stack(c["ctxs"], "lse"))) <= lt
+
+
+def test_scatter(case):
+    c = case
+    lh, pl, dt = c["lh"], c["pl"], c["dt"]
+    Og = _t(stack(c["ctxs"], "Og"), dt)
+    inv = _t(stack(c["ctxs"], "slot_of"), torch.int32)
+    O = lh.scatter(pl, Og, inv)
+    assert_close(np64(O), c["O"], dt, "O")
+
+
+def _grad_stack(c, key):
+    return np.stack([np.stack([g[key] for g in row]) for row in c["grads"][3]])
+
+
+def test_scatter_backward(case):
+    c = case
+    lh, pl, dt = c["lh"], c["pl"], c["dt"]
+    Og = _t(stack(c["ctxs"], "Og"), dt)
+    sel = _t(stack(c["ctxs"], "sel_idx"), torch.int32)
+    dOg, D = lh.scatter_bwd(pl, c["dO"], Og, sel)
+    assert_close(np64(dOg), _grad_stack(c, "dOg"), dt, "dOg")
+    assert_close(np64(D), _grad_stack(c, "D"), dt, "D")
+
+
+def test_attention_backward(case):
+    c = case
+    lh, dt = c["lh"], c["dt"]
+    Qg, Kg, Vg, Og = (_t(stack(c["ctxs"], k), dt) for k in ("Qg", "Kg", "Vg", "Og"))
+    lse = _t(stack(c["ctxs"], "lse"), torch.float32)
+    dOg = _t(_grad_stack(c, "dOg"), dt)
+    D = _t(_grad_stack(c, "D"), torch.float32)
+    for Din in (D, None):
+        dQg, dKg, dVg = lh.attn_bwd(Qg, Kg, Vg, Og, lse, dOg, Din)
+        assert_close(np64(dQg), _grad_stack(c, "dQg"), dt, "dQg")
+        assert_close(np64(dKg), _grad_stack(c, "dKg"), dt, "dKg")
+        assert_close(np64(dVg), _grad_stack(c, "dVg"), dt, "dVg")
+
+
+def test_gather_backward(case):
+    c = case
+    lh, pl, dt = c["lh"], c["pl"], c["dt"]
+    dXg = [_t(_grad_stack(c, k), dt) for k in ("dQg", "dKg", "dVg")]
+    inv = _t(stack(c["ctxs"], "slot_of"), torch.int32)
+    dQ, dK, dV = lh.gather_bwd(pl, *dXg, inv)
+    for got, exp, name in ((dQ, c["grads"][0], "dQ"), (dK, c["grads"][1], "dK"), (dV, c["grads"][2], "dV")):
+        assert_close(np64(got), exp, dt, name)
+
+
+def test_whole_layer(case):
+    c = case
+    lh, pl, dt = c["lh"], c["pl"], c["dt"]
+    O, ctx = lh.forward(pl, c["Q"], c["K"], c["V"])
+    dQ, dK, dV = lh.backward(pl, c["dO"], ctx)
+    torch.cuda.synchronize()
+    assert np.array_equal(ctx.sel_idx.cpu().numpy(), stack(c["ctxs"], "sel_idx"))
+    assert np.array_equal(ctx.slot_of.cpu().numpy(), stack(c["ctxs"], "slot_of"))
+    assert_close(np64(O), c["O"], dt, "O")
+    assert_close(np64(dQ), c["grads"][0], dt, "dQ")
+    assert_close(np64(dK), c["grads"][1], dt, "dK")
+    assert_close(np64(dV), c["grads"][2], dt, "dV")
+    # run to run: bit-identical
+    O2, ctx2 = lh.forward(pl, c["Q"], c["K"], c["V"])
+    g2 = lh.backward(pl, c["dO"], ctx2)
+    assert torch.equal(O, O2)
+    for a, b in zip((dQ, dK, dV), g2):
+        assert torch.equal(a, b)
+    lh.device_status()
+
+
+def test_dense_fixed_point_matches_attention():
+    """L = 1: the layer is plain causal attention on Q, K, V (skill card, 选择-注意力解耦)."""
+    from long_context_hierarchical_b200 import lh
+    Q, K, V, _ = make_inputs(1, 4, 1024, 64, "bf16", seed=3, device="cuda", with_grad=False)
+    pl = lh.plan(1, 4, 1024, 64, 4, 1, 0, "bf16")
+    O, _ = lh.forward(pl, Q, K, V)
+    Oa, _ = lh.attn_fwd(Q, K, V)
+    assert torch.equal(O, Oa)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q.float(), K.float(), V.float(), is_causal=True)
+    assert_close(np64(O), np64(ref), torch.bfloat16, "O vs SDPA")
