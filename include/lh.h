@@ -165,6 +165,29 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
                       const void* dOg, const float* D, void* dQg, void* dKg, void* dVg,
                       void* ws, size_t ws_bytes, lh_stream_t stream);
 
+/* Allocation-free variant of lh_attn_bwd (the paper has no counterpart; it
+ * exists for callers, not for the method).  Some callers hold only their
+ * input and output buffers and cannot allocate device memory: a kernel
+ * plug-in running inside another framework's engine with no allocator
+ * handle, or code on a path where a device allocation is not permitted.
+ * This entry point needs no workspace: the row term D = rowsum(dOg * Og) goes
+ * to a scratch array of LH_ATTN_BWD_STATIC_MAX_ROWS floats (4 MiB) compiled
+ * into the library, which every GPU that loads the library keeps until the
+ * process exits.  Same arguments and results as lh_attn_bwd with D = NULL.
+ *  - BH * S above LH_ATTN_BWD_STATIC_MAX_ROWS returns LH_ERR_WORKSPACE and
+ *    enqueues nothing.
+ *  - The first call on a device looks up the array's device address (a host
+ *    call, once per device); make that first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents:
+ *    calls whose work overlaps on the GPU (other streams, other threads) race
+ *    on it and must be serialised by the caller.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ *    call. */
+#define LH_ATTN_BWD_STATIC_MAX_ROWS (1 << 20)
+lh_status lh_attn_bwd_static(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
+                             const void* Kg, const void* Vg, const void* Og, const float* lse,
+                             const void* dOg, void* dQg, void* dKg, void* dVg, lh_stream_t stream);
+
 /* Stage 4 (skill card "阶段 4"; gist.science 2.C "deterministic scatter").
  * O[t] = sum over levels l (ascending) of Og[slot_of(l, floor((t+1)/p^l) - 1)]
  * where that index is >= 0 and selected; fp32 sum rounded once; 0 where no

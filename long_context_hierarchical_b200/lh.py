@@ -26,7 +26,7 @@ EXPORTS = (
     "lh_plan_init", "lh_pyramid", "lh_score", "lh_pyramid_score", "lh_topk", "lh_gather",
     "lh_attn_fwd", "lh_attn_bwd_ws_bytes", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd",
     "lh_gather_bwd", "lh_forward", "lh_backward", "lh_device_status", "lh_status_string",
-    "lh_last_error", "lh_plan_bytes",
+    "lh_last_error", "lh_plan_bytes", "lh_attn_bwd_static",
 )
 
 
@@ -81,6 +81,7 @@ def _load():
         "lh_forward": (PLAN, P, P, P, P, P, P, P),
         "lh_backward": (PLAN, P, P, P, P, P, P, P),
         "lh_device_status": (ctypes.c_int,),
+        "lh_attn_bwd_static": (I64, I64, I32, I32, P, P, P, P, P, P, P, P, P, P),
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -244,6 +245,18 @@ def attn_bwd(Qg, Kg, Vg, Og, lse, dOg, D=None, stream=None):
     _check(LIB.lh_attn_bwd(BH, S, d, code, _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(Og), _ptr(lse),
                            _ptr(dOg), _ptr(D), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(ws), ws.numel(),
                            _stream(stream)), "lh_attn_bwd")
+    return dQ, dK, dV
+
+
+def attn_bwd_static(Qg, Kg, Vg, Og, lse, dOg, stream=None):
+    """lh_attn_bwd with D computed into the library's own scratch array
+    (no workspace: for callers that cannot allocate device memory)."""
+    S, d = Qg.shape[-2], Qg.shape[-1]
+    BH = Qg.numel() // (S * d)
+    dQ, dK, dV = torch.empty_like(Qg), torch.empty_like(Kg), torch.empty_like(Vg)
+    _check(LIB.lh_attn_bwd_static(BH, S, d, _dtype_code(Qg), _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(Og),
+                                  _ptr(lse), _ptr(dOg), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                  _stream(stream)), "lh_attn_bwd_static")
     return dQ, dK, dV
 
 
