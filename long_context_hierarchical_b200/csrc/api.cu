@@ -257,6 +257,8 @@ static lh_status check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
   if (S >= (int64_t(1) << 31)) return fail(LH_ERR_INVALID_ARG, "S must stay below 2^31");
   if (dtype != LH_F32 && dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
   if (d != kD) return fail(LH_ERR_UNSUPPORTED, "only d = 64 is built");
+  if (dtype == LH_BF16 && BH > ((int64_t(1) << 31) - 1) / S)
+    return fail(LH_ERR_UNSUPPORTED, "bf16 attention needs BH * S < 2^31 (TMA row coordinates)");
   return LH_OK;
 }
 

@@ -10,8 +10,8 @@ cudaError_t launch_attn_bwd_f32(int64_t BH, int64_t S, const float* Q, const flo
                                 const float* D, float* dQ, float* dK, float* dV, cudaStream_t st);
 cudaError_t launch_rowdot(int64_t rows, int dtype, const void* dO, const void* O, float* D,
                           cudaStream_t st);
-cudaError_t launch_attn_fwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
-                                void* O, float* lse, cudaStream_t st);
+cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
+                               void* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                 const float* lse, const void* dO, const float* D, void* dQ,
                                 void* dK, void* dV, cudaStream_t st);
@@ -26,7 +26,7 @@ cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int dtype, const void* Qg, co
   if (dtype == LH_F32)
     return launch_attn_fwd_f32(BH, S, (const float*)Qg, (const float*)Kg, (const float*)Vg,
                                (float*)Og, lse, st);
-  return launch_attn_fwd_mma(BH, S, Qg, Kg, Vg, Og, lse, st);
+  return launch_attn_fwd_tc(BH, S, Qg, Kg, Vg, Og, lse, st);
 }
 
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,

@@ -1,10 +1,7 @@
-// Dense causal attention on the gathered sub-sequence, bf16 storage, on the
-// warp-level tensor-core path (mma.sync m16n8k16, fp32 accumulate).
-//
-// Stage 3 of the layer is ordinary causal softmax attention on [S, d]
-// (skill card "lighthouse-attention", stage 3; gist.science 2.C: stock
-// attention on a dense sub-sequence).  This file holds the backward pass,
-// and the forward used for the dense comparator's reference timing.
+// Backward of the dense causal attention on the gathered sub-sequence, bf16
+// storage, on the warp-level tensor-core path (mma.sync m16n8k16, fp32
+// accumulate).  Gradients flow through attention into the gathered rows
+// (skill card "lighthouse-attention", "梯度流").
 //
 // Tiles are 64 x 64 (queries x keys), d = 64, 4 warps per CTA, each warp
 // owning 16 rows of the CTA's tile.  K/V (or Q/dO) tiles are double-buffered
@@ -26,7 +23,6 @@ constexpr int kT = 64;       // tile rows / cols
 constexpr int kNT = 128;     // threads per CTA
 constexpr int kTileBytes = kT * kD * 2;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -150,100 +146,6 @@ __device__ __forceinline__ void store_rows(bf16* dst, int64_t r0, int64_t S, con
     if (r0 + g + 8 < S)
       *reinterpret_cast<uint32_t*>(dst + (r0 + g + 8) * kD + col) =
           pack_bf16(a[nb][2] * sb, a[nb][3] * sb);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// forward
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kNT)
-attn_fwd_mma_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K, const bf16* __restrict__ V,
-                    bf16* __restrict__ O, float* __restrict__ lse, int64_t S, int ntiles, float sl2) {
-  __shared__ __align__(128) uint8_t smem[5 * kTileBytes];
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK = sQ + kTileBytes, sV = sQ + 3 * kTileBytes;
-  const int qt = ntiles - 1 - blockIdx.x;  // long rows first
-  const int64_t bh = blockIdx.y;
-  const int64_t q0 = (int64_t)qt * kT;
-  const bf16* Qb = Q + bh * S * kD;
-  const bf16* Kb = K + bh * S * kD;
-  const bf16* Vb = V + bh * S * kD;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-
-  load_tile(sQ, Qb, q0, S);
-  load_tile(sK, Kb, 0, S);
-  load_tile(sV, Vb, 0, S);
-  cp_commit();
-
-  uint32_t qa[4][4];
-  float o[8][4];
-  zero(o);
-  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
-
-  for (int j = 0; j <= qt; ++j) {
-    const int buf = j & 1;
-    if (j + 1 <= qt) {
-      load_tile(sK + (buf ^ 1) * kTileBytes, Kb, (int64_t)(j + 1) * kT, S);
-      load_tile(sV + (buf ^ 1) * kTileBytes, Vb, (int64_t)(j + 1) * kT, S);
-    }
-    cp_commit();
-    cp_wait<1>();
-    __syncthreads();
-    if (j == 0) load_a_frags(sQ, warp * 16, qa);
-
-    float s[8][4];
-    zero(s);
-    mma_abt(s, qa, sK + buf * kTileBytes);
-
-    const bool diag = j == qt;
-    const int ra = warp * 16 + g, rb = ra + 8;
-    float mxa = -INFINITY, mxb = -INFINITY;
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = nb * 8 + 2 * t + (e & 1);
-        const int row = e < 2 ? ra : rb;
-        float v = s[nb][e] * sl2;
-        if (diag && col > row) v = -INFINITY;
-        s[nb][e] = v;
-        if (e < 2) mxa = fmaxf(mxa, v);
-        else mxb = fmaxf(mxb, v);
-      }
-    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
-    mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
-    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
-    mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-    const float na = fmaxf(ma, mxa), nbm = fmaxf(mb, mxb);
-    const float aa = exp2f(ma - na), ab = exp2f(mb - nbm);
-    float suma = 0.f, sumb = 0.f;
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      s[nb][0] = exp2f(s[nb][0] - na);
-      s[nb][1] = exp2f(s[nb][1] - na);
-      s[nb][2] = exp2f(s[nb][2] - nbm);
-      s[nb][3] = exp2f(s[nb][3] - nbm);
-      suma += s[nb][0] + s[nb][1];
-      sumb += s[nb][2] + s[nb][3];
-      o[nb][0] *= aa; o[nb][1] *= aa;
-      o[nb][2] *= ab; o[nb][3] *= ab;
-    }
-    la = la * aa + suma;
-    lb = lb * ab + sumb;
-    ma = na;
-    mb = nbm;
-    mma_pb(o, s, sV + buf * kTileBytes);
-    __syncthreads();
-  }
-  la += __shfl_xor_sync(0xffffffffu, la, 1);
-  la += __shfl_xor_sync(0xffffffffu, la, 2);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 1);
-  lb += __shfl_xor_sync(0xffffffffu, lb, 2);
-  const int64_t r0 = q0 + warp * 16;
-  store_rows(O + bh * S * kD, r0, S, o, 1.f / la, 1.f / lb);
-  if (t == 0) {
-    if (r0 + g < S) lse[bh * S + r0 + g] = (ma + log2f(la)) * kLn2;
-    if (r0 + g + 8 < S) lse[bh * S + r0 + g + 8] = (mb + log2f(lb)) * kLn2;
   }
 }
 
@@ -398,15 +300,6 @@ attn_bwd_dq_mma_kernel(const bf16* __restrict__ Q, const bf16* __restrict__ K,
 }
 
 }  // namespace
-
-cudaError_t launch_attn_fwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
-                                void* O, float* lse, cudaStream_t st) {
-  const int ntiles = (int)((S + kT - 1) / kT);
-  const float sl2 = 0.125f * kLog2e;
-  attn_fwd_mma_kernel<<<dim3(ntiles, (unsigned)BH), kNT, 0, st>>>(
-      (const bf16*)Q, (const bf16*)K, (const bf16*)V, (bf16*)O, lse, S, ntiles, sl2);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_attn_bwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                 const float* lse, const void* dO, const float* D, void* dQ,

@@ -1,0 +1,363 @@
+// Stage 3 forward on the 5th-generation tensor cores: causal attention on the
+// gathered [S, 64] bf16 sub-sequence (skill card "lighthouse-attention",
+// stage 3: a standard S x S causal mask; gist.science 2.C).
+//
+// One CTA owns 256 query rows as two 128-row tiles A and B and walks the key
+// tiles (128 keys) up to its diagonal.  Warp roles (320 threads):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
+//              query row r of its tile, which is TMEM lane r, so row max and
+//              row sum need no shuffles;
+//   warp 8     TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
+//   warp 9     TMEM allocation and the single MMA-issuing thread.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384),
+// fp32.  Per key tile j the MMA thread issues S_X = Q_X K_j^T (M=128, N=128,
+// 4 x K=16) and, once softmax X has written P_X (bf16, swizzled K-major smem),
+// O_X += P_X V_j (M=128, N=64, 8 x K=16, V read MN-major).  The two tiles
+// ping-pong so the tensor core works on one tile while the other's softmax
+// runs.  O is rescaled in TMEM only when a row maximum grows by more than
+// 2^8 (the reference maximum otherwise stays, so P <= 256).
+//
+// Every wait is bounded: on timeout the CTA records LH_ERR_TIMEOUT in the
+// device status word, stops issuing work, drains its own TMA copies and frees
+// its TMEM.
+#include <cudaTypedefs.h>
+
+#include "host.h"
+#include "tc.cuh"
+
+namespace lh {
+namespace {
+
+using bf16 = __nv_bfloat16;
+using namespace tc;
+
+constexpr int kRows = 128;                    // query rows per tile, keys per tile
+constexpr int kStages = 3;
+constexpr uint32_t kTile = kRows * kD * 2;    // 16 KB: 128 rows x 128 B
+constexpr uint32_t kPTile = kRows * kRows * 2;  // 32 KB
+constexpr int kThreads = 320;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescale = 8.0f;              // log2 units
+
+// Shared-memory map (offsets from a 1024-byte aligned base).
+constexpr uint32_t kOffQ = 0;                          // 2 tiles
+constexpr uint32_t kOffK = kOffQ + 2 * kTile;          // kStages tiles
+constexpr uint32_t kOffV = kOffK + kStages * kTile;    // kStages tiles
+constexpr uint32_t kOffP = kOffV + kStages * kTile;    // 2 P tiles
+constexpr uint32_t kOffBar = kOffP + 2 * kPTile;
+constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
+                   kBarS = kBarE + 8 * kStages, kBarP = kBarS + 16, kBarO = kBarP + 16,
+                   kBarDrain = kBarO + 16, kSlotTmem = kBarDrain + 8, kSlotAbort = kSlotTmem + 4;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+  // Bounded wait that ignores the abort flag (used to drain own copies).
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ O,
+                   float* __restrict__ lse, int S, int npairs, float sl2,
+                   unsigned int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + kOffBar;
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + kSlotAbort);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = npairs - 1 - (int)blockIdx.x;  // longest rows first
+  const int bh = blockIdx.y;
+  const int q0 = pair * 2 * kRows;
+  const int nA = 2 * pair + 1, nB = 2 * pair + 2;  // key tiles of tile A / tile B
+  const int row0 = bh * S;                          // first row of this head in the maps
+
+  if (threadIdx.x == 0) {
+    mbar_init(bars + kBarQ, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars + kBarK + 8 * s, 1);
+      mbar_init(bars + kBarV + 8 * s, 1);
+      mbar_init(bars + kBarE + 8 * s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bars + kBarS + 8 * x, 1);
+      mbar_init(bars + kBarP + 8 * x, 128);
+      mbar_init(bars + kBarO + 8 * x, 1);
+    }
+    mbar_init(bars + kBarDrain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) tmem_alloc(bars + kSlotTmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
+
+  if (warp == 8) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      mbar_expect_tx(bars + kBarQ, 2 * kTile);
+      tma_load_2d(base + kOffQ, &tmQ, 0, row0 + q0, bars + kBarQ);
+      tma_load_2d(base + kOffQ + kTile, &tmQ, 0, row0 + q0 + kRows, bars + kBarQ);
+      for (int j = 0; j < nB; ++j) {
+        const int s = j % kStages, u = j / kStages;
+        if (j >= kStages && !mbar_wait(bars + kBarE + 8 * s, (u - 1) & 1, abort, status)) break;
+        mbar_expect_tx(bars + kBarK + 8 * s, kTile);
+        tma_load_2d(base + kOffK + s * kTile, &tmK, 0, row0 + j * kRows, bars + kBarK + 8 * s);
+        mbar_expect_tx(bars + kBarV + 8 * s, kTile);
+        tma_load_2d(base + kOffV + s * kTile, &tmV, 0, row0 + j * kRows, bars + kBarV + 8 * s);
+        issued = j + 1;
+      }
+      if (*abort) {  // let this CTA's own copies land before its smem is released
+        wait_drain(bars + kBarQ, 0);
+        for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j) {
+          const int s = j % kStages, u = j / kStages;
+          wait_drain(bars + kBarK + 8 * s, u & 1);
+          wait_drain(bars + kBarV + 8 * s, u & 1);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kRows, kRows, false);
+      constexpr uint32_t idPV = idesc_bf16(kRows, kD, true);
+      auto issue_S = [&](int x, int j) {
+        const uint32_t q = base + kOffQ + x * kTile, k = base + kOffK + (j % kStages) * kTile;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_bf16(tmem + x * kRows, sw128_desc(q + ks * 32, 16, 1024),
+                   sw128_desc(k + ks * 32, 16, 1024), idS, ks > 0);
+      };
+      auto issue_PV = [&](int x, int j) {
+        const uint32_t p = base + kOffP + x * kPTile, v = base + kOffV + (j % kStages) * kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + 2 * kRows + x * kD,
+                   sw128_desc(p + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024),
+                   sw128_desc(v + kk * 2048, kTile, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bars + kBarQ, 0, abort, status) && mbar_wait(bars + kBarK, 0, abort, status);
+      if (ok) {
+        tc_fence_after();
+        issue_S(0, 0);
+        mma_commit(bars + kBarS);
+        issue_S(1, 0);
+        mma_commit(bars + kBarS + 8);
+      }
+      for (int j = 0; ok && j < nB; ++j) {
+        const int s = j % kStages, u = j / kStages;
+        const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
+        bool v_ready = false;
+        if (j < nA) {
+          if (!(ok = mbar_wait(bars + kBarP, j & 1, abort, status))) break;
+          if (!(ok = mbar_wait(bars + kBarV + 8 * s, u & 1, abort, status))) break;
+          v_ready = true;
+          tc_fence_after();
+          issue_PV(0, j);
+          if (j + 1 < nA) {
+            if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
+            issue_S(0, j + 1);
+            mma_commit(bars + kBarS);
+          } else {
+            mma_commit(bars + kBarO);
+          }
+        }
+        if (!(ok = mbar_wait(bars + kBarP + 8, j & 1, abort, status))) break;
+        if (!v_ready && !(ok = mbar_wait(bars + kBarV + 8 * s, u & 1, abort, status))) break;
+        tc_fence_after();
+        issue_PV(1, j);
+        if (j + 1 < nB) {
+          if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
+          issue_S(1, j + 1);
+          mma_commit(bars + kBarS + 8);
+        } else {
+          mma_commit(bars + kBarO + 8);
+        }
+        mma_commit(bars + kBarE + 8 * s);  // K_j and V_j free once these MMAs are done
+      }
+      // Every MMA issued here has finished before TMEM is released.
+      mma_commit(bars + kBarDrain);
+      wait_drain(bars + kBarDrain, 0);
+    }
+  } else {
+    // ---------------- softmax, one query row per thread ----------------
+    const int x = warp >> 2, wr = warp & 3;
+    const int r = wr * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
+    const uint32_t tS = lane_base + x * kRows, tO = lane_base + 2 * kRows + x * kD;
+    const int n = x ? nB : nA;
+    const int qrow = q0 + x * kRows + r;
+    const uint32_t prow = base + kOffP + x * kPTile + r * 128;
+    float m_ref = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f);  // row sum, two partial sums
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      ok = mbar_wait(bars + kBarS + 8 * x, j & 1, abort, status);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before TMEM access
+      tc_fence_after();
+      const bool diag = j == n - 1;
+      // Keys after this query (only on the diagonal tile) are masked.
+      const int lim = diag ? qrow - j * kRows : kRows;  // columns < lim are visible
+      // Pass 1: row maximum of the raw scores (sl2 > 0 keeps the order).
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        float a[32], b[32];
+        tmem_ld32(tS + 64 * c2, a);
+        tmem_ld32(tS + 64 * c2 + 32, b);
+        tmem_wait_ld();
+        if (diag) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (64 * c2 + e > lim) a[e] = -INFINITY;
+            if (64 * c2 + 32 + e > lim) b[e] = -INFINITY;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) mx = max3f(mx, fmax3f(a[e], a[e + 1], b[e]), b[e + 1]);
+      }
+      mx *= sl2;
+      const float m_new = mx > m_ref + kRescale ? mx : m_ref;
+      const float alpha = exp2f(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
+      if (j > 0 && __any_sync(0xffffffffu, m_new != m_ref)) {
+        float o[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tO + 32 * c, o);
+        }
+        tmem_wait_st();
+      }
+      m_ref = m_new;
+      l2.x *= alpha;
+      l2.y *= alpha;
+      // Pass 2: P = 2^(s*sl2 - m_ref), row sum, bf16 P into the swizzled tile.
+      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_wait_ld();
+        if (diag) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * c + e > lim) v[e] = -INFINITY;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float2 t = ffma2(make_float2(v[e], v[e + 1]), sc2, nm2);
+          t.x = ex2_approx(t.x);
+          t.y = ex2_approx(t.y);
+          l2 = fadd2(l2, t);
+          w[e >> 1] = pack_bf16x2(t.x, t.y);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int ch = c * 4 + q;  // 16-byte chunk of the 256-byte row
+          const uint32_t dst = prow + (ch >> 3) * (kRows * 128) + (((ch & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(w[4 * q]),
+                       "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bars + kBarP + 8 * x);
+    }
+    const float l = l2.x + l2.y;
+    if (ok) ok = mbar_wait(bars + kBarO + 8 * x, 0, abort, status);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      float o[2][32];
+      tmem_ld32(tO, o[0]);
+      tmem_ld32(tO + 32, o[1]);
+      tmem_wait_ld();
+      if (qrow < S) {
+        const float inv = 1.f / l;
+        bf16* dst = O + ((int64_t)row0 + qrow) * kD;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int col = c * 8 + 2 * h;
+            __nv_bfloat162 b2 =
+                __floats2bfloat162_rn(o[col >> 5][col & 31] * inv, o[(col + 1) >> 5][(col + 1) & 31] * inv);
+            w[h] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        lse[(int64_t)row0 + qrow] = (m_ref + log2f(l)) * kLn2;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// [rows, 64] bf16 row-major, tiles of 128 rows x 64 columns, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kRows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
+                               void* O, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, Q, BH * S) || !make_tile_map(&mk, K, BH * S) ||
+      !make_tile_map(&mv, V, BH * S))
+    return cudaErrorInvalidValue;
+  unsigned int* status = device_status_ptr();
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int npairs = (int)((S + 2 * kRows - 1) / (2 * kRows));
+  const float sl2 = 0.125f * 1.4426950408889634f;
+  attn_fwd_tc_kernel<<<dim3(npairs, (unsigned)BH), kThreads, kSmemBytes, st>>>(
+      mq, mk, mv, static_cast<bf16*>(O), lse, (int)S, npairs, sl2, status);
+  return cudaGetLastError();
+}
+
+}  // namespace lh

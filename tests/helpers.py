@@ -62,7 +62,9 @@ def grad_term_bounds(Qg, Kg, Vg, Og, lse, dOg):
     roundings reach the terms on the GPU: the bf16 operand dS of the MMA and
     the bf16 storage of Og, which enters D_i = sum_c dOg_ic Og_ic.  Per term
     the bound used is P_ij (|dP_ij| + sum_c |dOg_ic Og_ic|) times |Kg_j| (or
-    |Qg_i|); dVg_j = sum_i P_ij dOg_i gets P_ij |dOg_i|.
+    |Qg_i|); dVg_j = sum_i P_ij dOg_i gets P_ij |dOg_i|.  The forward output
+    Og_i = sum_j P_ij Vg_j (P rounded to bf16 for the MMA on the GPU) gets
+    sum_j P_ij |Vg_j|.
     """
     S, d = Qg.shape
     scale = 1.0 / np.sqrt(d)
@@ -70,7 +72,8 @@ def grad_term_bounds(Qg, Kg, Vg, Og, lse, dOg):
     mq = np.zeros_like(Qg)
     mk = np.zeros_like(Kg)
     mv = np.zeros_like(Vg)
-    aK, aQ, aG = np.abs(Kg), np.abs(Qg), np.abs(dOg)
+    mo = np.zeros_like(Vg)
+    aK, aQ, aG, aV = np.abs(Kg), np.abs(Qg), np.abs(dOg), np.abs(Vg)
     for r0 in range(0, S, 512):
         r1 = min(S, r0 + 512)
         s = (Qg[r0:r1] @ Kg[:r1].T) * scale
@@ -82,27 +85,32 @@ def grad_term_bounds(Qg, Kg, Vg, Og, lse, dOg):
         mq[r0:r1] = (T @ aK[:r1]) * scale
         mk[:r1] += (T.T @ aQ[r0:r1]) * scale
         mv[:r1] += P.T @ aG[r0:r1]
-    return mq, mk, mv
+        mo[r0:r1] = P @ aV[:r1]
+    return mq, mk, mv, mo
 
 
 def grad_tolerance_terms(ctxs, grads, sz):
     """Per-element term bounds of dQ/dK/dV (gathered and per token), all heads."""
-    out = {k: [] for k in ("dQg", "dKg", "dVg", "dQ", "dK", "dV")}
+    out = {k: [] for k in ("dQg", "dKg", "dVg", "dQ", "dK", "dV", "Og", "O")}
     for crow, grow in zip(ctxs, grads[3]):
         r = {k: [] for k in out}
         for ctx, g in zip(crow, grow):
-            mq, mk, mv = grad_term_bounds(ctx["Qg"], ctx["Kg"], ctx["Vg"], ctx["Og"], ctx["lse"], g["dOg"])
+            mq, mk, mv, mo = grad_term_bounds(ctx["Qg"], ctx["Kg"], ctx["Vg"], ctx["Og"], ctx["lse"],
+                                              g["dOg"])
             for key, m in (("dQ", mq), ("dK", mk), ("dV", mv)):
                 r[key + "g"].append(m)
                 r[key].append(oracle.gather_bwd(m, ctx["slot_of"], sz, "f64"))
+            r["Og"].append(mo)
+            r["O"].append(oracle.scatter(mo, ctx["slot_of"], sz, "f64"))
         for k in out:
             out[k].append(np.stack(r[k]))
     return {k: np.stack(v) for k, v in out.items()}
 
 
 def assert_grad_close(got, exp, terms, dtype, what):
-    """Gradient check: TOL * max(1, |exp|) plus one bf16 rounding step (2^-7)
-    of the sum of |terms| (``grad_term_bounds``); fp32 uses 2^-23."""
+    """Check of a cancelling sum (attention output or gradient): TOL * max(1,
+    |exp|) plus one bf16 rounding step (2^-7) of the sum of |terms|
+    (``grad_term_bounds``); fp32 uses 2^-23."""
     got = np.asarray(got, dtype=np.float64)
     exp = np.asarray(exp, dtype=np.float64)
     step = 2.0 ** -7 if dtype == torch.bfloat16 else 2.0 ** -23
