@@ -12,9 +12,9 @@ cudaError_t launch_rowdot(int64_t rows, int dtype, const void* dO, const void* O
                           cudaStream_t st);
 cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                void* O, float* lse, cudaStream_t st);
-cudaError_t launch_attn_bwd_mma(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
-                                const float* lse, const void* dO, const float* D, void* dQ,
-                                void* dK, void* dV, cudaStream_t st);
+cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
+                               const float* lse, const void* dO, const float* D, void* dQ,
+                               void* dK, void* dV, cudaStream_t st);
 
 int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype) {
   (void)dtype;
@@ -42,7 +42,7 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, co
   if (dtype == LH_F32)
     return launch_attn_bwd_f32(BH, S, (const float*)Qg, (const float*)Kg, (const float*)Vg, lse,
                                (const float*)dOg, D, (float*)dQg, (float*)dKg, (float*)dVg, st);
-  return launch_attn_bwd_mma(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, st);
+  return launch_attn_bwd_tc(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, st);
 }
 
 }  // namespace lh
