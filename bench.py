@@ -22,7 +22,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import torch
@@ -66,7 +65,7 @@ class ClockSampler:
             self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.tmp, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -296,10 +295,26 @@ def dense_sdpa_ms(H, N, steps=3, backward=True):
     return a.elapsed_time(b) / steps
 
 
+def workload_extras(w, fwd_ms, fb_ms, dense_steps=3):
+    """Forward / forward+backward throughput and dense causal SDPA at the same N."""
+    out = {"fwd_ms": fwd_ms, "fwd_bwd_ms": fb_ms,
+           "fwd_mtok_s": w.B * w.N / (fwd_ms * 1e-3) / 1e6,
+           "fwd_bwd_mtok_s": w.B * w.N / (fb_ms * 1e-3) / 1e6}
+    try:
+        sd_f = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False)
+        sd_fb = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True)
+        out["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb,
+                                   "speedup_fwd": sd_f / fwd_ms, "speedup_fwd_bwd": sd_fb / fb_ms}
+    except Exception as e:  # comparator only
+        out["dense_sdpa_torch"] = {"error": str(e)[:200]}
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="lighthouse", choices=["lighthouse", "reference"])
     ap.add_argument("--workload", default="98k_k1536", choices=list(WORKLOADS))
@@ -406,16 +421,22 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         fwd_ms, _ = timed_steps(layer, stp, args.steps, backward=False)
-        extras["fwd_mtok_s"] = w.B * w.N / (fwd_ms * 1e-3) / 1e6
-        extras["fwd_ms"] = fwd_ms
-        try:
-            sd_f = dense_sdpa_ms(w.H, w.N, backward=False)
-            sd_fb = dense_sdpa_ms(w.H, w.N, backward=True)
-            extras["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb,
-                                          "speedup_fwd": sd_f / fwd_ms, "speedup_fwd_bwd": sd_fb / ms}
-        except Exception as e:  # comparator only
-            extras["dense_sdpa_torch"] = {"error": str(e)[:200]}
+        extras[w.name] = workload_extras(w, fwd_ms, ms)
+        del layer, Q, K, V, dO, hQ, hK, hV, hdO, hO, hdQ, hdK, hdV, dQ, dK, dV, O
         torch.cuda.empty_cache()
+        if w.name != "512k_k2048":
+            w5 = WORKLOADS["512k_k2048"]
+            Q5, K5, V5, dO5 = make_workload_inputs(w5, seed=0, device="cuda")
+            l5 = Layer(lh, w5, Q5, K5, V5, dO5)
+            for _ in range(2):
+                l5.step(stp)
+            torch.cuda.synchronize()
+            fb5, st5 = timed_steps(l5, stp, 3)
+            f5, _ = timed_steps(l5, stp, 3, backward=False)
+            extras[w5.name] = workload_extras(w5, f5, fb5, dense_steps=1)
+            extras[w5.name]["stages_ms"] = dict(zip(STAGES, st5))
+            del l5, Q5, K5, V5, dO5
+            torch.cuda.empty_cache()
         Qh, Kh, Vh, dOh = cpu_sample_inputs(w, 0, 0)
         secs = oracle_head_seconds(w, Qh, Kh, Vh, dOh)
         heads = w.B * w.H

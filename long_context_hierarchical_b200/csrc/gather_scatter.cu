@@ -68,6 +68,26 @@ gather_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K, const T* 
 }
 
 template <typename T>
+__device__ __forceinline__ void store_stream(T* p, const float (&x)[8]);
+template <>
+__device__ __forceinline__ void store_stream<__nv_bfloat16>(__nv_bfloat16* p, const float (&x)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&h);
+  }
+  __stcs(reinterpret_cast<uint4*>(p), make_uint4(w[0], w[1], w[2], w[3]));
+}
+template <>
+__device__ __forceinline__ void store_stream<float>(float* p, const float (&x)[8]) {
+  __stcs(reinterpret_cast<float4*>(p), make_float4(x[0], x[1], x[2], x[3]));
+  __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
+}
+
+// L is a template parameter so the per-level index loads and row loads are
+// all issued before the first one is used.
+template <typename T, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
@@ -78,20 +98,29 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
   const int64_t t = row - bh * g.N;
   const int32_t* inv = slot_of + bh * g.Ntot;
   const T* og = Og + bh * g.S * kD + c * 8;
+  int32_t slot[L];
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    const int64_t i = ((t + 1) >> (g.logp * l)) - 1;
+    slot[l] = i >= 0 ? __ldg(inv + g.flat_off[l] + i) : -1;
+  }
+  float x[L][8];
+#pragma unroll
+  for (int l = 0; l < L; ++l) {
+    if (slot[l] >= 0 && slot[l] < g.S) Vec8<T>::load(og + (int64_t)slot[l] * kD, x[l]);
+    else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[l][e] = 0.f;
+    }
+  }
   float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int l = 0; l < g.L; ++l) {
-    const int64_t i = ((t + 1) >> (g.logp * l)) - 1;
-    if (i < 0) break;  // coarser levels start later still
-    const int32_t slot = __ldg(inv + g.flat_off[l] + i);
-    if (slot < 0 || slot >= g.S) continue;
-    float x[8];
-    Vec8<T>::load(og + (int64_t)slot * kD, x);
+  for (int e = 0; e < 8; ++e) {
+    acc[e] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += x[e];
+    for (int l = 0; l < L; ++l) acc[e] += x[l][e];  // ascending level
   }
-  Vec8<T>::store(O + row * kD + c * 8, acc);
+  store_stream<T>(O + row * kD + c * 8, acc);
 }
 
 template <typename T>
@@ -133,7 +162,7 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   if (c == 0) D[r] = dsum;
 }
 
-template <typename T>
+template <typename T, int L>
 __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
@@ -145,30 +174,32 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   const int64_t t = row - bh * g.N;
   const int32_t* inv = slot_of + bh * g.Ntot;
   const int64_t base = bh * g.S * kD + c * 8;
-  float aq[8], ak[8], av[8];
+  int32_t slot[L];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = av[e] = 0.f;
-  for (int l = 0; l < g.L; ++l) {
-    const int sh = g.logp * l;
-    const int32_t slot = __ldg(inv + g.flat_off[l] + (t >> sh));
-    if (slot < 0 || slot >= g.S) continue;
-    const float w = 1.f / (float)(1 << sh);  // exact: a power of two
-    const int64_t o = base + (int64_t)slot * kD;
-    float x[8];
-    Vec8<T>::load(dQg + o, x);
+  for (int l = 0; l < L; ++l) slot[l] = __ldg(inv + g.flat_off[l] + (t >> (g.logp * l)));
+  const T* src[3] = {dQg, dKg, dVg};
+  T* dst[3] = {dQ, dK, dV};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) aq[e] = fmaf(x[e], w, aq[e]);
-    Vec8<T>::load(dKg + o, x);
+  for (int w = 0; w < 3; ++w) {
+    float x[L][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ak[e] = fmaf(x[e], w, ak[e]);
-    Vec8<T>::load(dVg + o, x);
+    for (int l = 0; l < L; ++l) {
+      if (slot[l] >= 0 && slot[l] < g.S) Vec8<T>::load(src[w] + base + (int64_t)slot[l] * kD, x[l]);
+      else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) av[e] = fmaf(x[e], w, av[e]);
+        for (int e = 0; e < 8; ++e) x[l][e] = 0.f;
+      }
+    }
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      acc[e] = 0.f;
+#pragma unroll
+      for (int l = 0; l < L; ++l)  // ascending level; 1/p^l is a power of two: exact
+        acc[e] = fmaf(x[l][e], 1.f / (float)(1 << (g.logp * l)), acc[e]);
+    }
+    store_stream<T>(dst[w] + row * kD + c * 8, acc);
   }
-  const int64_t out = row * kD + c * 8;
-  Vec8<T>::store(dQ + out, aq);
-  Vec8<T>::store(dK + out, ak);
-  Vec8<T>::store(dV + out, av);
 }
 
 unsigned blocks_for(int64_t rows) { return (unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock); }
@@ -194,15 +225,28 @@ cudaError_t launch_gather(const lh_plan& plan, const void* Q, const void* K, con
   return cudaGetLastError();
 }
 
+template <typename T, int L>
+void scatter_l(const Geo& g, unsigned b, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
+  scatter_kernel<T, L><<<b, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+}
+
+template <typename T>
+void scatter_t(const Geo& g, unsigned b, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
+  switch (g.L) {
+    case 1: scatter_l<T, 1>(g, b, Og, slot_of, O, st); break;
+    case 2: scatter_l<T, 2>(g, b, Og, slot_of, O, st); break;
+    case 3: scatter_l<T, 3>(g, b, Og, slot_of, O, st); break;
+    case 4: scatter_l<T, 4>(g, b, Og, slot_of, O, st); break;
+    default: scatter_l<T, 5>(g, b, Og, slot_of, O, st); break;
+  }
+}
+
 cudaError_t launch_scatter(const lh_plan& plan, const void* Og, const int32_t* slot_of, void* O,
                            cudaStream_t st) {
   const Geo g = make_geo(plan);
   const unsigned b = blocks_for(g.BH * g.N);
-  if (plan.c.dtype == LH_BF16)
-    scatter_kernel<__nv_bfloat16><<<b, kThreads, 0, st>>>(g, (const __nv_bfloat16*)Og, slot_of,
-                                                          (__nv_bfloat16*)O);
-  else
-    scatter_kernel<float><<<b, kThreads, 0, st>>>(g, (const float*)Og, slot_of, (float*)O);
+  if (plan.c.dtype == LH_BF16) scatter_t<__nv_bfloat16>(g, b, Og, slot_of, O, st);
+  else scatter_t<float>(g, b, Og, slot_of, O, st);
   return cudaGetLastError();
 }
 
@@ -220,20 +264,32 @@ cudaError_t launch_scatter_bwd(const lh_plan& plan, const void* dO, const void* 
   return cudaGetLastError();
 }
 
+template <typename T, int L>
+void gather_bwd_l(const Geo& g, unsigned b, const void* dQg, const void* dKg, const void* dVg,
+                  const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
+  gather_bwd_kernel<T, L><<<b, kThreads, 0, st>>>(g, (const T*)dQg, (const T*)dKg, (const T*)dVg,
+                                                  slot_of, (T*)dQ, (T*)dK, (T*)dV);
+}
+
+template <typename T>
+void gather_bwd_t(const Geo& g, unsigned b, const void* dQg, const void* dKg, const void* dVg,
+                  const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
+  switch (g.L) {
+    case 1: gather_bwd_l<T, 1>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
+    case 2: gather_bwd_l<T, 2>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
+    case 3: gather_bwd_l<T, 3>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
+    case 4: gather_bwd_l<T, 4>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
+    default: gather_bwd_l<T, 5>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
+  }
+}
+
 cudaError_t launch_gather_bwd(const lh_plan& plan, const void* dQg, const void* dKg,
                               const void* dVg, const int32_t* slot_of, void* dQ, void* dK,
                               void* dV, cudaStream_t st) {
   const Geo g = make_geo(plan);
   const unsigned b = blocks_for(g.BH * g.N);
-  if (plan.c.dtype == LH_BF16) {
-    using T = __nv_bfloat16;
-    gather_bwd_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)dQg, (const T*)dKg, (const T*)dVg,
-                                                 slot_of, (T*)dQ, (T*)dK, (T*)dV);
-  } else {
-    using T = float;
-    gather_bwd_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)dQg, (const T*)dKg, (const T*)dVg,
-                                                 slot_of, (T*)dQ, (T*)dK, (T*)dV);
-  }
+  if (plan.c.dtype == LH_BF16) gather_bwd_t<__nv_bfloat16>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
+  else gather_bwd_t<float>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
   return cudaGetLastError();
 }
 

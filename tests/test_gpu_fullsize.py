@@ -1,0 +1,163 @@
+"""Parity at the full benchmark sizes (98K and 512K tokens, 16 heads, bf16).
+
+The layer runs on the GPU exactly as the benchmark runs it (lh_forward /
+lh_backward on the whole [1, 16, N, 64] problem).  The oracle then checks
+sampled heads: pyramid levels, scores and the selection in full; the
+attention output at sampled tokens (through the oracle's attention rows of
+the slots that reach them); and, at 98K with k = 1536, dQ/dK/dV on a
+4096-token prefix (oracle backward restricted to the slots that reach the
+prefix, with the full forward's LSE and D).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import lighthouse as oracle
+from long_context_hierarchical_b200.synth import WORKLOADS, make_workload_inputs
+from tests.helpers import assert_pyr_close, np64
+
+pytestmark = pytest.mark.gpu
+
+HEADS = (0, 11)           # sampled (b=0) heads
+N_TOKENS = 192            # sampled output tokens per head
+PREFIX = 4096             # gradient prefix
+
+
+def _bf16(x):
+    return oracle.round_bf16(x)
+
+
+def _attention_rows_with_bounds(Qg, Kg, Vg, rows):
+    """Oracle output rows plus sum_j P_ij |Vg_j| (the cancelling-sum bound)."""
+    O, lse = oracle.attention_rows(Qg, Kg, Vg, rows)
+    d = Qg.shape[1]
+    T = np.empty_like(O)
+    aV = np.abs(Vg)
+    for a, r in enumerate(rows):
+        s = (Kg[: r + 1] @ Qg[r]) / np.sqrt(d)
+        P = np.exp(s - lse[a])
+        T[a] = P @ aV[: r + 1]
+    return O, lse, T
+
+
+def _check(got, exp, terms, what):
+    err = np.abs(got - exp)
+    tol = 2e-2 * np.maximum(1.0, np.abs(exp)) + 2.0 ** -7 * terms
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
+                           f"max abs err {err.max():.3e}")
+
+
+@pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048"])
+def run(request):
+    from long_context_hierarchical_b200 import lh
+    w = WORKLOADS[request.param]
+    Q, K, V, dO = make_workload_inputs(w, seed=0, device="cuda")
+    pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+    O, ctx = lh.forward(pl, Q, K, V)
+    grads = lh.backward(pl, dO, ctx) if request.param == "98k_k1536" else None
+    pyr, scores = lh.pyramid_score(pl, Q, K, V)
+    torch.cuda.synchronize()
+    lh.device_status()
+    yield dict(w=w, lh=lh, pl=pl, Q=Q, K=K, V=V, dO=dO, O=O, ctx=ctx, grads=grads, pyr=pyr,
+               scores=scores)
+    del Q, K, V, dO, O, ctx, grads, pyr, scores
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("h", HEADS)
+def test_fullsize_selection_and_output(run, h):
+    w, pl, ctx = run["w"], run["pl"], run["ctx"]
+    sz = oracle.sizes(w.N, w.p, w.L, w.k)
+    Qh, Kh, Vh = (np64(run[x][0, h]) for x in ("Q", "K", "V"))
+    # scores and selection, in full
+    cand, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz)
+    got_scores = np64(run["scores"][0, h])
+    assert np.max(np.abs(got_scores - cand) / np.maximum(cand, 1e-30)) <= 1e-6
+    assert np.array_equal(ctx.sel_idx[0, h].cpu().numpy(), sel_idx)
+    assert np.array_equal(ctx.slot_of[0, h].cpu().numpy(), slot_of)
+    # pyramid levels, in full (one rounding step plus the fp32 summation bound)
+    levels = [oracle.pyramid(X, sz, "bf16") for X in (Qh, Kh, Vh)]
+    for t, X in enumerate((Qh, Kh, Vh)):
+        exp = np.concatenate(levels[t][1:], axis=0)
+        absmean = np.concatenate(oracle.pyramid(np.abs(X), sz, "f64")[1:], axis=0)
+        span = np.concatenate([np.full(sz.n[l], sz.P[l]) for l in range(1, sz.L)])
+        assert_pyr_close(np64(run["pyr"][t][0, h]), exp, torch.bfloat16, f"pyramid[{t}]", absmean, span)
+    # the gathered rows are the selected pyramid entries
+    Qg, Kg, Vg = (oracle.gather(levels[t], sel_idx, sz) for t in range(3))
+    for name, exp in (("Qg", Qg), ("Kg", Kg), ("Vg", Vg)):
+        got = np64(ctx.gathered(name)[0, h])
+        assert np.all(np.abs(got - exp) <= 2.0 ** -7 * np.abs(exp) + 1e-4), name
+    # output at sampled tokens (first, last and spread), via the slots reaching them
+    rng = np.random.default_rng(h)
+    tokens = np.unique(np.concatenate([[0, 1, sz.P[-1] - 1, w.N - 1],
+                                       rng.integers(0, w.N, N_TOKENS)]))
+    need = set()
+    for t in tokens:
+        for l in range(sz.L):
+            i = (t + 1) // sz.P[l] - 1
+            if i >= 0 and slot_of[sz.flat_off[l] + i] >= 0:
+                need.add(int(slot_of[sz.flat_off[l] + i]))
+    need = sorted(need)
+    Orows, lse_rows, Trows = _attention_rows_with_bounds(Qg, Kg, Vg, need)
+    Og = {j: _bf16(Orows[a]) for a, j in enumerate(need)}
+    Tg = {j: Trows[a] for a, j in enumerate(need)}
+    got_lse = np64(ctx.lse[0, h])[need]
+    assert np.max(np.abs(got_lse - lse_rows)) <= 1e-3
+    exp_O = np.zeros((tokens.size, w.d))
+    term = np.zeros((tokens.size, w.d))
+    for a, t in enumerate(tokens):
+        for l in range(sz.L):
+            i = (t + 1) // sz.P[l] - 1
+            if i >= 0 and slot_of[sz.flat_off[l] + i] >= 0:
+                j = int(slot_of[sz.flat_off[l] + i])
+                exp_O[a] += Og[j]
+                term[a] += Tg[j]
+    _check(np64(run["O"][0, h])[tokens], _bf16(exp_O), term, f"O[{w.name}, head {h}]")
+
+
+def test_fullsize_gradient_prefix(run):
+    """dQ, dK, dV on tokens t < 4096 of one head (98K, k = 1536)."""
+    if run["grads"] is None:
+        pytest.skip("gradients are checked on the 98K k=1536 workload")
+    w, ctx = run["w"], run["ctx"]
+    h = HEADS[1]
+    sz = oracle.sizes(w.N, w.p, w.L, w.k)
+    Qh, Kh, Vh, dOh = (np64(run[x][0, h]) for x in ("Q", "K", "V", "dO"))
+    _, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz)
+    levels = [oracle.pyramid(X, sz, "bf16") for X in (Qh, Kh, Vh)]
+    Qg, Kg, Vg = (oracle.gather(levels[t], sel_idx, sz) for t in range(3))
+    Og_exact, lse = oracle.causal_attention(Qg, Kg, Vg)
+    Og = _bf16(Og_exact)
+    dOg = oracle.scatter_bwd(dOh, sel_idx, sz, "bf16")
+    D = np.sum(dOg * Og, axis=1)
+    scale = 1.0 / np.sqrt(w.d)
+    # slots whose span starts before the prefix end
+    lev, idx = oracle.entry_level_index(sel_idx, sz)
+    J = np.nonzero(idx * np.asarray(sz.P)[lev] < PREFIX)[0]
+    jmax = int(J.max()) + 1
+    # dQg rows J (row-local)
+    s = (Qg[J] @ Kg[:jmax].T) * scale
+    P = np.where(np.arange(jmax)[None, :] <= J[:, None], np.exp(s - lse[J, None]), 0.0)
+    dP = dOg[J] @ Vg[:jmax].T
+    dS = P * (dP - D[J, None])
+    A = np.sum(np.abs(dOg * Og), axis=1)
+    dQg = np.zeros_like(Qg)
+    tQg = np.zeros_like(Qg)
+    dQg[J] = (dS @ Kg[:jmax]) * scale
+    tQg[J] = ((P * (np.abs(dP) + A[J, None])) @ np.abs(Kg[:jmax])) * scale
+    # dKg, dVg columns J (all query rows at or after each key)
+    s = (Qg @ Kg[J].T) * scale
+    P = np.where(np.arange(sz.S)[:, None] >= J[None, :], np.exp(s - lse[:, None]), 0.0)
+    dP = dOg @ Vg[J].T
+    dS = P * (dP - D[:, None])
+    dKg, dVg, tKg, tVg = (np.zeros_like(Qg) for _ in range(4))
+    dKg[J] = (dS.T @ Qg) * scale
+    dVg[J] = P.T @ dOg
+    tKg[J] = ((P * (np.abs(dP) + A[:, None])).T @ np.abs(Qg)) * scale
+    tVg[J] = P.T @ np.abs(dOg)
+    got = [np64(g[0, h][:PREFIX]) for g in run["grads"]]
+    for g, dXg, tX, name in zip(got, (dQg, dKg, dVg), (tQg, tKg, tVg), ("dQ", "dK", "dV")):
+        exp = oracle.gather_bwd(_bf16(dXg), slot_of, sz, "bf16")[:PREFIX]
+        term = oracle.gather_bwd(tX, slot_of, sz, "f64")[:PREFIX]
+        _check(g, exp, term, f"{name} prefix")
