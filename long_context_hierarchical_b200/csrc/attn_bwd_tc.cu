@@ -18,6 +18,10 @@
 // needed here), warp 8 loads (TMA for tiles, plain loads for LSE/D), warp 9
 // owns TMEM and issues the MMAs from one thread.  TMEM columns: [0,128) S or
 // S^T, [128,256) dP or dP^T, [256,320) dQ or dV, [320,384) dK.
+// Overlap: each element-wise thread copies its S/dP columns out of TMEM and
+// releases them at once, so the next tile's S and dP MMAs run while it
+// computes; the single P/dS shared-memory tile has its own "consumed"
+// barrier that the element-wise warps wait on just before overwriting it.
 // Operand layouts are those of the forward kernel: K-major A/B tiles with the
 // 128-byte swizzle, tiles read as the MN-major B operand (dO, Q, K) with
 // 8-row groups 1024 bytes apart.  Every wait is bounded (see tc.cuh).
@@ -90,7 +94,8 @@ constexpr uint32_t kOffVec = kOffDST + kWide;            // kStages x (128 lse2 
 constexpr uint32_t kOffBar = kOffVec + kStages * 1024;
 constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * kStages,
                    kBarSP = kBarEmpty + 8 * kStages, kBarPDS = kBarSP + 8, kBarAcc = kBarPDS + 8,
-                   kBarDrain = kBarAcc + 8, kSlotTmem = kBarDrain + 8, kSlotAbort = kSlotTmem + 4;
+                   kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8, kBarPF = kBarTF + 8,
+                   kSlotTmem = kBarPF + 8, kSlotAbort = kSlotTmem + 4;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 }  // namespace kv
 
@@ -126,6 +131,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     mbar_init(bars + kBarPDS, 256);
     mbar_init(bars + kBarAcc, 1);
     mbar_init(bars + kBarDrain, 1);
+    mbar_init(bars + kBarTF, 256);  // S^T/dP^T copied out of TMEM
+    mbar_init(bars + kBarPF, 1);    // P^T/dS^T tile consumed by the MMAs
     *abort = 0;
     fence_mbar_init();
   }
@@ -197,21 +204,24 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       }
       for (int t = 0; ok && t < nq; ++t) {
         const int s = t % kStages;
-        if (!(ok = mbar_wait(bars + kBarPDS, t & 1, abort, status))) break;
+        // S^T/dP^T of tile t copied out: start tile t+1's while tile t computes
+        if (!(ok = mbar_wait(bars + kBarTF, t & 1, abort, status))) break;
         tc_fence_after();
-        gemm_acc(tmem + 2 * kRows, base + kOffPT, base + kOffG + s * kTile, t > 0);       // dV += P^T dO
-        gemm_acc(tmem + 2 * kRows + kD, base + kOffDST, base + kOffQ + s * kTile, t > 0); // dK += dS^T Q
-        mma_commit(bars + kBarEmpty + 8 * s);
         if (t + 1 < nq) {
           const int s1 = (t + 1) % kStages, u1 = (t + 1) / kStages;
           if (!(ok = mbar_wait(bars + kBarFull + 8 * s1, u1 & 1, abort, status))) break;
           gemm_sq(tmem, base + kOffK, base + kOffQ + s1 * kTile);
           gemm_sq(tmem + kRows, base + kOffV, base + kOffG + s1 * kTile);
           mma_commit(bars + kBarSP);
-        } else {
-          mma_commit(bars + kBarAcc);
         }
+        if (!(ok = mbar_wait(bars + kBarPDS, t & 1, abort, status))) break;
+        tc_fence_after();
+        gemm_acc(tmem + 2 * kRows, base + kOffPT, base + kOffG + s * kTile, t > 0);       // dV += P^T dO
+        gemm_acc(tmem + 2 * kRows + kD, base + kOffDST, base + kOffQ + s * kTile, t > 0); // dK += dS^T Q
+        mma_commit(bars + kBarPF);
+        mma_commit(bars + kBarEmpty + 8 * s);
       }
+      if (ok) mma_commit(bars + kBarAcc);
       mma_commit(bars + kBarDrain);
       wait_drain(bars + kBarDrain, 0);
     }
@@ -234,33 +244,43 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       const bool edge = (t == 0) || (q0 + kRows > S);
       const float* l2 = vec + s * 256;
       const float* dd = l2 + 128;
+      float st[2][32], dp[2][32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(lane_base + half * 64 + c * 32, st[c]);
+        tmem_ld32(lane_base + kRows + half * 64 + c * 32, dp[c]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
+      uint32_t wp[2][16], wd[2][16];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int col0 = half * 64 + c * 32;
-        float st[32], dp[32];
-        tmem_ld32(lane_base + col0, st);
-        tmem_ld32(lane_base + kRows + col0, dp);
-        tmem_wait_ld();
-        uint32_t wp[16], wd[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const float4 lv = *reinterpret_cast<const float4*>(l2 + col0 + (e & ~3));
           const float4 dv = *reinterpret_cast<const float4*>(dd + col0 + (e & ~3));
           const float la = (e & 2) ? lv.z : lv.x, lb = (e & 2) ? lv.w : lv.y;
           const float da = (e & 2) ? dv.z : dv.x, db = (e & 2) ? dv.w : dv.y;
-          float2 x = ffma2(make_float2(st[e], st[e + 1]), sc2, make_float2(-la, -lb));
+          float2 x = ffma2(make_float2(st[c][e], st[c][e + 1]), sc2, make_float2(-la, -lb));
           float pa = ex2_approx(x.x), pb = ex2_approx(x.y);
           if (edge) {
             const int qa = q0 + col0 + e;
             if (qa < key || qa >= S) pa = 0.f;
             if (qa + 1 < key || qa + 1 >= S) pb = 0.f;
           }
-          const float dsa = pa * (dp[e] - da), dsb = pb * (dp[e + 1] - db);
-          wp[e >> 1] = pack_bf16x2(pa, pb);
-          wd[e >> 1] = pack_bf16x2(dsa, dsb);
+          wp[c][e >> 1] = pack_bf16x2(pa, pb);
+          wd[c][e >> 1] = pack_bf16x2(pa * (dp[c][e] - da), pb * (dp[c][e + 1] - db));
         }
-        store_row32(base + kOffPT, r, half * 2 + c, wp);
-        store_row32(base + kOffDST, r, half * 2 + c, wd);
+      }
+      // the previous tile's P^T / dS^T must be consumed before they are overwritten
+      if (t > 0) ok = mbar_wait(bars + kBarPF, (t - 1) & 1, abort, status);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        store_row32(base + kOffPT, r, half * 2 + c, wp[c]);
+        store_row32(base + kOffDST, r, half * 2 + c, wd[c]);
       }
       fence_proxy_async();
       tc_fence_before();
@@ -299,7 +319,8 @@ constexpr uint32_t kOffDS = kOffV + kStages * kTile;   // dS (128 x 128)
 constexpr uint32_t kOffBar = kOffDS + kWide;
 constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
                    kBarSP = kBarE + 8 * kStages, kBarDS = kBarSP + 8, kBarAcc = kBarDS + 8,
-                   kBarDrain = kBarAcc + 8, kSlotTmem = kBarDrain + 8, kSlotAbort = kSlotTmem + 4;
+                   kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8, kBarDF = kBarTF + 8,
+                   kSlotTmem = kBarDF + 8, kSlotAbort = kSlotTmem + 4;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 }  // namespace qq
 
@@ -335,6 +356,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     mbar_init(bars + kBarDS, 256);
     mbar_init(bars + kBarAcc, 1);
     mbar_init(bars + kBarDrain, 1);
+    mbar_init(bars + kBarTF, 256);  // S/dP copied out of TMEM
+    mbar_init(bars + kBarDF, 1);    // dS tile consumed by the MMA
     *abort = 0;
     fence_mbar_init();
   }
@@ -386,14 +409,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       }
       for (int j = 0; ok && j < nk; ++j) {
         const int s = j % kStages;
-        if (!(ok = mbar_wait(bars + kBarDS, j & 1, abort, status))) break;
+        if (!(ok = mbar_wait(bars + kBarTF, j & 1, abort, status))) break;
         tc_fence_after();
-        const uint32_t kk_tile = base + kOffK + s * kTile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dQ += dS K
-          mma_bf16(tmem + 2 * kRows, sw128_desc(base + kOffDS + (kk >> 2) * kKBlock + (kk & 3) * 32, 16, 1024),
-                   sw128_desc(kk_tile + kk * 2048, kTile, 1024), idAcc, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars + kBarE + 8 * s);
         if (j + 1 < nk) {
           const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
           if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
@@ -401,10 +418,18 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
           gemm_sq(tmem, base + kOffQ, base + kOffK + s1 * kTile);
           gemm_sq(tmem + kRows, base + kOffG, base + kOffV + s1 * kTile);
           mma_commit(bars + kBarSP);
-        } else {
-          mma_commit(bars + kBarAcc);
         }
+        if (!(ok = mbar_wait(bars + kBarDS, j & 1, abort, status))) break;
+        tc_fence_after();
+        const uint32_t kk_tile = base + kOffK + s * kTile;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // dQ += dS K
+          mma_bf16(tmem + 2 * kRows, sw128_desc(base + kOffDS + (kk >> 2) * kKBlock + (kk & 3) * 32, 16, 1024),
+                   sw128_desc(kk_tile + kk * 2048, kTile, 1024), idAcc, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bars + kBarDF);
+        mma_commit(bars + kBarE + 8 * s);
       }
+      if (ok) mma_commit(bars + kBarAcc);
       mma_commit(bars + kBarDrain);
       wait_drain(bars + kBarDrain, 0);
     }
@@ -423,26 +448,34 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       tc_fence_after();
       const bool diag = j == nk - 1;
       const int lim = qrow - j * kRows;  // visible columns: c <= lim
+      float sv[2][32], dp[2][32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32(lane_base + half * 64 + c * 32, sv[c]);
+        tmem_ld32(lane_base + kRows + half * 64 + c * 32, dp[c]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
+      uint32_t w[2][16];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const int col0 = half * 64 + c * 32;
-        float sv[32], dp[32];
-        tmem_ld32(lane_base + col0, sv);
-        tmem_ld32(lane_base + kRows + col0, dp);
-        tmem_wait_ld();
-        uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float2 x = ffma2(make_float2(sv[e], sv[e + 1]), sc2, nl2);
+          float2 x = ffma2(make_float2(sv[c][e], sv[c][e + 1]), sc2, nl2);
           float pa = ex2_approx(x.x), pb = ex2_approx(x.y);
           if (diag) {
             if (col0 + e > lim) pa = 0.f;
             if (col0 + e + 1 > lim) pb = 0.f;
           }
-          w[e >> 1] = pack_bf16x2(pa * (dp[e] - Dr), pb * (dp[e + 1] - Dr));
+          w[c][e >> 1] = pack_bf16x2(pa * (dp[c][e] - Dr), pb * (dp[c][e + 1] - Dr));
         }
-        store_row32(base + kOffDS, r, half * 2 + c, w);
       }
+      if (j > 0) ok = mbar_wait(bars + kBarDF, (j - 1) & 1, abort, status);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) store_row32(base + kOffDS, r, half * 2 + c, w[c]);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(bars + kBarDS);
