@@ -13,10 +13,10 @@
 //  - dq: one CTA per 128-query tile walks the key tiles up to its diagonal.
 //    S = Q K^T and dP = dO V^T in TMEM (lane = query), dS to smem,
 //    dQ += dS K in TMEM.
-// Warp roles (320 threads): warps 0-3 and 4-7 are two element-wise groups
-// that split the 128 columns of each tile in halves (no row reductions are
-// needed here), warp 8 loads (TMA for tiles, plain loads for LSE/D), warp 9
-// owns TMEM and issues the MMAs from one thread.  TMEM columns: [0,128) S or
+// Warp roles (576 threads): warps 0-15 are four element-wise groups of four
+// warps that split the 128 columns of each tile in quarters (no row
+// reductions are needed here), warp 16 loads (TMA for tiles, plain loads for
+// LSE/D), warp 17 owns TMEM and issues the MMAs from one thread.  TMEM columns: [0,128) S or
 // S^T, [128,256) dP or dP^T, [256,320) dQ or dV, [320,384) dK.
 // Overlap: each element-wise thread copies its S/dP columns out of TMEM and
 // releases them at once, so the next tile's S and dP MMAs run while it
@@ -42,7 +42,10 @@ constexpr int kStages = 3;
 constexpr uint32_t kTile = kRows * kD * 2;      // 16 KB
 constexpr uint32_t kKBlock = kRows * 128;       // one 64-column K-block of a 128-wide tile
 constexpr uint32_t kWide = 2 * kKBlock;         // 32 KB: 128 x 128 bf16
-constexpr int kThreads = 320;
+constexpr int kGroups = 4;                      // element-wise warp groups
+constexpr int kEw = kGroups * 128;              // element-wise threads
+constexpr int kLoadWarp = 4 * kGroups, kMmaWarp = kLoadWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
@@ -128,21 +131,21 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       mbar_init(bars + kBarEmpty + 8 * s, 1);
     }
     mbar_init(bars + kBarSP, 1);
-    mbar_init(bars + kBarPDS, 256);
+    mbar_init(bars + kBarPDS, kEw);
     mbar_init(bars + kBarAcc, 1);
     mbar_init(bars + kBarDrain, 1);
-    mbar_init(bars + kBarTF, 256);  // S^T/dP^T copied out of TMEM
+    mbar_init(bars + kBarTF, kEw);  // S^T/dP^T copied out of TMEM
     mbar_init(bars + kBarPF, 1);    // P^T/dS^T tile consumed by the MMAs
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(bars + kSlotTmem, 512);
+  if (warp == kMmaWarp) tmem_alloc(bars + kSlotTmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
 
-  if (warp == 8) {
+  if (warp == kLoadWarp) {
     // ---------------- loads ----------------
     int issued = 0;
     if (lane == 0) {
@@ -177,7 +180,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
         wait_drain(bars + kBarFull + 8 * (t % kStages), (t / kStages) & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idSq = idesc_bf16(kRows, kRows, false);
@@ -227,9 +230,10 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     }
   } else {
     // ---------------- element-wise: P^T, dS^T ----------------
-    const int half = warp >> 2, wr = warp & 3;
+    const int grp = warp >> 2, wr = warp & 3;
     const int r = wr * 32 + lane;  // key row of the tile = TMEM lane
     const int key = k0 + r;
+    const int col0 = grp * 32;     // this group's 32 query columns
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = true;
@@ -242,67 +246,60 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       const int q0 = (kt + t) * kRows;
       // visible: key <= query < S
       const bool edge = (t == 0) || (q0 + kRows > S);
-      const float* l2 = vec + s * 256;
+      const float* l2 = vec + s * 256 + col0;
       const float* dd = l2 + 128;
-      float st[2][32], dp[2][32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(lane_base + half * 64 + c * 32, st[c]);
-        tmem_ld32(lane_base + kRows + half * 64 + c * 32, dp[c]);
-      }
+      float st[32], dp[32];
+      tmem_ld32(lane_base + col0, st);
+      tmem_ld32(lane_base + kRows + col0, dp);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
-      uint32_t wp[2][16], wd[2][16];
+      uint32_t wp[16], wd[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int col0 = half * 64 + c * 32;
+      for (int e = 0; e < 32; e += 4) {
+        const float4 lv = *reinterpret_cast<const float4*>(l2 + e);
+        const float4 dv = *reinterpret_cast<const float4*>(dd + e);
+        float2 x0 = ffma2(make_float2(st[e], st[e + 1]), sc2, make_float2(-lv.x, -lv.y));
+        float2 x1 = ffma2(make_float2(st[e + 2], st[e + 3]), sc2, make_float2(-lv.z, -lv.w));
+        float p[4] = {ex2_approx(x0.x), ex2_approx(x0.y), ex2_approx(x1.x), ex2_approx(x1.y)};
+        if (edge) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float4 lv = *reinterpret_cast<const float4*>(l2 + col0 + (e & ~3));
-          const float4 dv = *reinterpret_cast<const float4*>(dd + col0 + (e & ~3));
-          const float la = (e & 2) ? lv.z : lv.x, lb = (e & 2) ? lv.w : lv.y;
-          const float da = (e & 2) ? dv.z : dv.x, db = (e & 2) ? dv.w : dv.y;
-          float2 x = ffma2(make_float2(st[c][e], st[c][e + 1]), sc2, make_float2(-la, -lb));
-          float pa = ex2_approx(x.x), pb = ex2_approx(x.y);
-          if (edge) {
-            const int qa = q0 + col0 + e;
-            if (qa < key || qa >= S) pa = 0.f;
-            if (qa + 1 < key || qa + 1 >= S) pb = 0.f;
+          for (int u = 0; u < 4; ++u) {
+            const int qa = q0 + col0 + e + u;
+            if (qa < key || qa >= S) p[u] = 0.f;
           }
-          wp[c][e >> 1] = pack_bf16x2(pa, pb);
-          wd[c][e >> 1] = pack_bf16x2(pa * (dp[c][e] - da), pb * (dp[c][e + 1] - db));
         }
+        wp[e >> 1] = pack_bf16x2(p[0], p[1]);
+        wp[(e >> 1) + 1] = pack_bf16x2(p[2], p[3]);
+        wd[e >> 1] = pack_bf16x2(p[0] * (dp[e] - dv.x), p[1] * (dp[e + 1] - dv.y));
+        wd[(e >> 1) + 1] = pack_bf16x2(p[2] * (dp[e + 2] - dv.z), p[3] * (dp[e + 3] - dv.w));
       }
       // the previous tile's P^T / dS^T must be consumed before they are overwritten
       if (t > 0) ok = mbar_wait(bars + kBarPF, (t - 1) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        store_row32(base + kOffPT, r, half * 2 + c, wp[c]);
-        store_row32(base + kOffDST, r, half * 2 + c, wd[c]);
-      }
+      store_row32(base + kOffPT, r, grp, wp);
+      store_row32(base + kOffDST, r, grp, wd);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(bars + kBarPDS);
     }
     if (ok) ok = mbar_wait(bars + kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
+      // groups 0,1: dV columns [32 grp, +32); groups 2,3: dK columns [32 (grp-2), +32)
       tc_fence_after();
-      float v[32], k[32];
-      tmem_ld32(lane_base + 2 * kRows + half * 32, v);
-      tmem_ld32(lane_base + 2 * kRows + kD + half * 32, k);
+      const bool isk = grp >= 2;
+      const int c = (grp & 1) * 32;
+      float v[32];
+      tmem_ld32(lane_base + 2 * kRows + (isk ? kD : 0) + c, v);
       tmem_wait_ld();
-      if (key < S) {
-        store_out32(dV + ((int64_t)row0 + key) * kD + half * 32, v, 1.f);
-        store_out32(dK + ((int64_t)row0 + key) * kD + half * 32, k, scale);
-      }
+      if (key < S)
+        store_out32((isk ? dK : dV) + ((int64_t)row0 + key) * kD + c, v, isk ? scale : 1.f);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -353,21 +350,21 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       mbar_init(bars + kBarE + 8 * s, 1);
     }
     mbar_init(bars + kBarSP, 1);
-    mbar_init(bars + kBarDS, 256);
+    mbar_init(bars + kBarDS, kEw);
     mbar_init(bars + kBarAcc, 1);
     mbar_init(bars + kBarDrain, 1);
-    mbar_init(bars + kBarTF, 256);  // S/dP copied out of TMEM
+    mbar_init(bars + kBarTF, kEw);  // S/dP copied out of TMEM
     mbar_init(bars + kBarDF, 1);    // dS tile consumed by the MMA
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(bars + kSlotTmem, 512);
+  if (warp == kMmaWarp) tmem_alloc(bars + kSlotTmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
 
-  if (warp == 8) {
+  if (warp == kLoadWarp) {
     if (lane == 0) {
       int issued = 0;
       mbar_expect_tx(bars + kBarQ, 2 * kTile);
@@ -390,7 +387,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idSq = idesc_bf16(kRows, kRows, false);
       constexpr uint32_t idAcc = idesc_bf16(kRows, kD, true);
@@ -434,9 +431,10 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       wait_drain(bars + kBarDrain, 0);
     }
   } else {
-    const int half = warp >> 2, wr = warp & 3;
+    const int grp = warp >> 2, wr = warp & 3;
     const int r = wr * 32 + lane;
     const int qrow = q0 + r;
+    const int col0 = grp * 32;  // this group's 32 key columns
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
     const float l2 = qrow < S ? lse[row0 + qrow] * kLog2e : 0.f;
     const float Dr = qrow < S ? Dv[row0 + qrow] : 0.f;
@@ -447,52 +445,44 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
       const bool diag = j == nk - 1;
-      const int lim = qrow - j * kRows;  // visible columns: c <= lim
-      float sv[2][32], dp[2][32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32(lane_base + half * 64 + c * 32, sv[c]);
-        tmem_ld32(lane_base + kRows + half * 64 + c * 32, dp[c]);
-      }
+      const int lim = qrow - j * kRows - col0;  // visible columns of this group: c <= lim
+      float sv[32], dp[32];
+      tmem_ld32(lane_base + col0, sv);
+      tmem_ld32(lane_base + kRows + col0, dp);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
-      uint32_t w[2][16];
+      uint32_t w[16];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int col0 = half * 64 + c * 32;
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float2 x = ffma2(make_float2(sv[c][e], sv[c][e + 1]), sc2, nl2);
-          float pa = ex2_approx(x.x), pb = ex2_approx(x.y);
-          if (diag) {
-            if (col0 + e > lim) pa = 0.f;
-            if (col0 + e + 1 > lim) pb = 0.f;
-          }
-          w[c][e >> 1] = pack_bf16x2(pa * (dp[c][e] - Dr), pb * (dp[c][e + 1] - Dr));
+      for (int e = 0; e < 32; e += 2) {
+        float2 x = ffma2(make_float2(sv[e], sv[e + 1]), sc2, nl2);
+        float pa = ex2_approx(x.x), pb = ex2_approx(x.y);
+        if (diag) {
+          if (e > lim) pa = 0.f;
+          if (e + 1 > lim) pb = 0.f;
         }
+        w[e >> 1] = pack_bf16x2(pa * (dp[e] - Dr), pb * (dp[e + 1] - Dr));
       }
       if (j > 0) ok = mbar_wait(bars + kBarDF, (j - 1) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) store_row32(base + kOffDS, r, half * 2 + c, w[c]);
+      store_row32(base + kOffDS, r, grp, w);
       fence_proxy_async();
       tc_fence_before();
       mbar_arrive(bars + kBarDS);
     }
     if (ok) ok = mbar_wait(bars + kBarAcc, 0, abort, status);
-    if (__all_sync(0xffffffffu, ok)) {
+    if (__all_sync(0xffffffffu, ok) && grp < 2) {
       tc_fence_after();
       float v[32];
-      tmem_ld32(lane_base + 2 * kRows + half * 32, v);
+      tmem_ld32(lane_base + 2 * kRows + grp * 32, v);
       tmem_wait_ld();
-      if (qrow < S) store_out32(dQ + ((int64_t)row0 + qrow) * kD + half * 32, v, scale);
+      if (qrow < S) store_out32(dQ + ((int64_t)row0 + qrow) * kD + grp * 32, v, scale);
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
