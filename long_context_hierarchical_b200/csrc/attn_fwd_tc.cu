@@ -3,12 +3,14 @@
 // stage 3: a standard S x S causal mask; gist.science 2.C).
 //
 // One CTA owns 256 query rows as two 128-row tiles A and B and walks the key
-// tiles (128 keys) up to its diagonal.  Warp roles (320 threads):
-//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
-//              query row r of its tile, which is TMEM lane r, so row max and
-//              row sum need no shuffles;
-//   warp 8     TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
-//   warp 9     TMEM allocation and the single MMA-issuing thread.
+// tiles (128 keys) up to its diagonal.  Warp roles (576 threads):
+//   warps 0-7  softmax of tile A, warps 8-15 softmax of tile B, each tile's
+//              eight warps as two groups on column halves [0,64), [64,128):
+//              thread r of a group owns query row r of its tile (TMEM lane
+//              r), so a row's max and sum need no shuffles, only one
+//              exchange of the two halves' maxima through shared memory;
+//   warp 16    TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
+//   warp 17    TMEM allocation and the single MMA-issuing thread.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384),
 // fp32.  Per key tile j the MMA thread issues S_X = Q_X K_j^T (M=128, N=128,
 // 4 x K=16) and, once softmax X has written P_X (bf16, swizzled K-major smem),
@@ -35,7 +37,8 @@ constexpr int kRows = 128;                    // query rows per tile, keys per t
 constexpr int kStages = 3;
 constexpr uint32_t kTile = kRows * kD * 2;    // 16 KB: 128 rows x 128 B
 constexpr uint32_t kPTile = kRows * kRows * 2;  // 32 KB
-constexpr int kThreads = 320;
+constexpr int kLoadWarp = 16, kMmaWarp = 17;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;              // log2 units
 
@@ -47,8 +50,13 @@ constexpr uint32_t kOffP = kOffV + kStages * kTile;    // 2 P tiles
 constexpr uint32_t kOffBar = kOffP + 2 * kPTile;
 constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
                    kBarS = kBarE + 8 * kStages, kBarP = kBarS + 16, kBarO = kBarP + 16,
-                   kBarDrain = kBarO + 16, kSlotTmem = kBarDrain + 8, kSlotAbort = kSlotTmem + 4;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
+                   kBarDrain = kBarO + 16, kBarRed = kBarDrain + 8, kBarL = kBarRed + 32,
+                   kSlotTmem = kBarL + 16, kSlotAbort = kSlotTmem + 4;
+// Row-max exchange between the two column halves: [parity][tile][half][row];
+// then the row-sum exchange: [tile][half][row].
+constexpr uint32_t kOffRed = kOffBar + 256;
+constexpr uint32_t kOffL = kOffRed + 2 * 2 * 2 * kRows * 4;
+constexpr uint32_t kSmemBytes = kOffL + 2 * 2 * kRows * 4 + 1024;  // + alignment slack
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   // Bounded wait that ignores the abort flag (used to drain own copies).
@@ -86,20 +94,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bars + kBarS + 8 * x, 1);
-      mbar_init(bars + kBarP + 8 * x, 128);
+      mbar_init(bars + kBarP + 8 * x, 256);
       mbar_init(bars + kBarO + 8 * x, 1);
+      mbar_init(bars + kBarRed + 16 * x, 256);
+      mbar_init(bars + kBarRed + 16 * x + 8, 256);
+      mbar_init(bars + kBarL + 8 * x, 256);
     }
     mbar_init(bars + kBarDrain, 1);
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tmem_alloc(bars + kSlotTmem, 512);
+  if (warp == kMmaWarp) tmem_alloc(bars + kSlotTmem, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
 
-  if (warp == 8) {
+  if (warp == kLoadWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int issued = 0;
@@ -124,7 +135,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kRows, kRows, false);
@@ -188,76 +199,82 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       wait_drain(bars + kBarDrain, 0);
     }
   } else {
-    // ---------------- softmax, one query row per thread ----------------
-    const int x = warp >> 2, wr = warp & 3;
+    // ---------------- softmax, one query row per thread, half the columns ----------------
+    const int x = warp >> 3, h = (warp >> 2) & 1, wr = warp & 3;
     const int r = wr * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
-    const uint32_t tS = lane_base + x * kRows, tO = lane_base + 2 * kRows + x * kD;
+    const uint32_t tS = lane_base + x * kRows + 64 * h, tO = lane_base + 2 * kRows + x * kD + 32 * h;
     const int n = x ? nB : nA;
     const int qrow = q0 + x * kRows + r;
-    const uint32_t prow = base + kOffP + x * kPTile + r * 128;
+    const uint32_t prow = base + kOffP + x * kPTile + h * (kRows * 128) + r * 128;
+    float* red = reinterpret_cast<float*>(gbase + kOffRed);
+    float* lsum = reinterpret_cast<float*>(gbase + kOffL);
     float m_ref = -INFINITY;
-    float2 l2 = make_float2(0.f, 0.f);  // row sum, two partial sums
+    float2 l2 = make_float2(0.f, 0.f);  // this half's row sum, two partial sums
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       ok = mbar_wait(bars + kBarS + 8 * x, j & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before TMEM access
       tc_fence_after();
       const bool diag = j == n - 1;
-      // Keys after this query (only on the diagonal tile) are masked.
-      const int lim = diag ? qrow - j * kRows : kRows;  // columns < lim are visible
-      // Pass 1: row maximum of the raw scores (sl2 > 0 keeps the order).
+      // Keys after this query (only on the diagonal tile) are masked:
+      // columns c of this half with 64 h + c > lim.
+      const int lim = diag ? qrow - j * kRows - 64 * h : kRows;
+      float v[2][32];
+      tmem_ld32(tS, v[0]);
+      tmem_ld32(tS + 32, v[1]);
+      tmem_wait_ld();
+      if (diag) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (e > lim) v[0][e] = -INFINITY;
+          if (32 + e > lim) v[1][e] = -INFINITY;
+        }
+      }
+      // Row maximum of the raw scores over this half (sl2 > 0 keeps the
+      // order), then over both halves through shared memory.
       float mx = -INFINITY;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        float a[32], b[32];
-        tmem_ld32(tS + 64 * c2, a);
-        tmem_ld32(tS + 64 * c2 + 32, b);
-        tmem_wait_ld();
-        if (diag) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (64 * c2 + e > lim) a[e] = -INFINITY;
-            if (64 * c2 + 32 + e > lim) b[e] = -INFINITY;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) mx = max3f(mx, fmax3f(a[e], a[e + 1], b[e]), b[e + 1]);
-      }
-      mx *= sl2;
+      for (int e = 0; e < 32; e += 2) mx = max3f(mx, fmax3f(v[0][e], v[0][e + 1], v[1][e]), v[1][e + 1]);
+      float* rj = red + ((j & 1) * 4 + x * 2) * kRows;
+      rj[h * kRows + r] = mx;
+      mbar_arrive(bars + kBarRed + 16 * x + 8 * (j & 1));
+      ok = mbar_wait(bars + kBarRed + 16 * x + 8 * (j & 1), (j >> 1) & 1, abort, status);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      mx = fmaxf(mx, rj[(h ^ 1) * kRows + r]) * sl2;
       const float m_new = mx > m_ref + kRescale ? mx : m_ref;
       const float alpha = exp2f(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
       if (j > 0 && __any_sync(0xffffffffu, m_new != m_ref)) {
         float o[32];
+        tmem_ld32(tO, o);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(tO + 32 * c, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(tO + 32 * c, o);
-        }
+        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+        tmem_st32(tO, o);
         tmem_wait_st();
       }
       m_ref = m_new;
       l2.x *= alpha;
       l2.y *= alpha;
-      // Pass 2: P = 2^(s*sl2 - m_ref), row sum, bf16 P into the swizzled tile.
+      // P = 2^(s*sl2 - m_ref), row sum, bf16 P into this half's K-block.
+      // S is read from TMEM again rather than kept live across the exchange.
+      tmem_ld32(tS, v[0]);
+      tmem_ld32(tS + 32, v[1]);
+      tmem_wait_ld();
+      if (diag) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (e > lim) v[0][e] = -INFINITY;
+          if (32 + e > lim) v[1][e] = -INFINITY;
+        }
+      }
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tS + 32 * c, v);
-        tmem_wait_ld();
-        if (diag) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * c + e > lim) v[e] = -INFINITY;
-        }
+      for (int c = 0; c < 2; ++c) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          float2 t = ffma2(make_float2(v[e], v[e + 1]), sc2, nm2);
+          float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
           t.x = ex2_approx(t.x);
           t.y = ex2_approx(t.y);
           l2 = fadd2(l2, t);
@@ -265,8 +282,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int ch = c * 4 + q;  // 16-byte chunk of the 256-byte row
-          const uint32_t dst = prow + (ch >> 3) * (kRows * 128) + (((ch & 7) ^ (r & 7)) << 4);
+          const int ch = c * 4 + q;  // 16-byte chunk within this half's 128-byte row
+          const uint32_t dst = prow + ((ch ^ (r & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(w[4 * q]),
                        "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
                        : "memory");
@@ -276,37 +293,37 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_before();
       mbar_arrive(bars + kBarP + 8 * x);
     }
-    const float l = l2.x + l2.y;
+    // Row sum over both halves.
+    if (ok) {
+      lsum[(x * 2 + h) * kRows + r] = l2.x + l2.y;
+      mbar_arrive(bars + kBarL + 8 * x);
+      ok = mbar_wait(bars + kBarL + 8 * x, 0, abort, status);
+    }
     if (ok) ok = mbar_wait(bars + kBarO + 8 * x, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
+      const float l = lsum[(x * 2) * kRows + r] + lsum[(x * 2 + 1) * kRows + r];
       tc_fence_after();
-      float o[2][32];
-      tmem_ld32(tO, o[0]);
-      tmem_ld32(tO + 32, o[1]);
+      float o[32];
+      tmem_ld32(tO, o);
       tmem_wait_ld();
       if (qrow < S) {
         const float inv = 1.f / l;
-        bf16* dst = O + ((int64_t)row0 + qrow) * kD;
+        bf16* dst = O + ((int64_t)row0 + qrow) * kD + 32 * h;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t w[4];
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const int col = c * 8 + 2 * h;
-            __nv_bfloat162 b2 =
-                __floats2bfloat162_rn(o[col >> 5][col & 31] * inv, o[(col + 1) >> 5][(col + 1) & 31] * inv);
-            w[h] = *reinterpret_cast<uint32_t*>(&b2);
-          }
+          for (int q = 0; q < 4; ++q) w[q] = pack_bf16x2(o[8 * c + 2 * q] * inv, o[8 * c + 2 * q + 1] * inv);
           reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        lse[(int64_t)row0 + qrow] = (m_ref + log2f(l)) * kLn2;
+        if (h == 0) lse[(int64_t)row0 + qrow] = (m_ref + log2f(l)) * kLn2;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/lh.h"
+#include "lh.h"
 
 namespace lh {
 

@@ -6,7 +6,7 @@
 
 #include <string>
 
-#include "../../include/lh.h"
+#include "lh.h"
 #include "common.cuh"
 
 namespace lh {
