@@ -105,27 +105,6 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&d);
 }
 
-// 2^x on the FMA pipe, for x in [-inf, 64]: Cody-Waite style reduction
-// x = n + f, n = round(x) (the 1.5 * 2^23 shift leaves n in the low mantissa
-// bits), f in [-1/2, 1/2], 2^f by a degree-3 minimax polynomial in relative
-// error (Remez exchange; coefficients from gen_exp2_poly.py, max relative
-// error 7.5e-5), and 2^n added to the exponent field.  Inputs below -125 are
-// clamped there, giving 2^-125 instead of a smaller value.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 shift = make_float2(12582912.f, 12582912.f);
-  const float2 c0 = make_float2(0.99992806f, 0.99992806f), c1 = make_float2(0.69326097f, 0.69326097f);
-  const float2 c2 = make_float2(0.24261113f, 0.24261113f), c3 = make_float2(0.05517167f, 0.05517167f);
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, shift);
-  const float2 f = fsub2(x, fsub2(t, shift));
-  float2 p = ffma2(f, c3, c2);
-  p = ffma2(p, f, c1);
-  p = ffma2(p, f, c0);
-  const int nx = __float_as_int(t.x) << 23, ny = __float_as_int(t.y) << 23;
-  return make_float2(__int_as_float(__float_as_int(p.x) + nx), __int_as_float(__float_as_int(p.y) + ny));
-}
-
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
