@@ -50,18 +50,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises *abort, records LH_ERR_TIMEOUT in *status) if it does not within
-// kWaitCycles, or at once if *abort is already raised.
+// kWaitCycles, or soon after *abort is raised elsewhere (checked every 64
+// polls, which keeps the shared-memory traffic of waiting threads down).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (true) {
-    if (*abort) return false;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitCycles) {
-      *abort = 1;
-      if (status) atomicExch(status, 5u /* LH_ERR_TIMEOUT */);
-      return false;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort = 1;
+        if (status) atomicExch(status, 5u /* LH_ERR_TIMEOUT */);
+        return false;
+      }
     }
   }
 }
