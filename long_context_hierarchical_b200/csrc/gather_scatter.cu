@@ -85,67 +85,78 @@ __device__ __forceinline__ void store_stream<float>(float* p, const float (&x)[8
   __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(x[4], x[5], x[6], x[7]));
 }
 
-// L is a template parameter so the per-level index loads and row loads are
-// all issued before the first one is used.
-template <typename T, int L>
+// p = 2^LOGP and L are template parameters, the head comes from blockIdx.y
+// and indices inside a head are 32-bit, so the per-token index arithmetic is
+// a handful of shifts and adds.
+template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
-  const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
+  const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
   const int c = threadIdx.x & 7;
-  if (row >= g.BH * g.N) return;
-  const int64_t bh = row / g.N;
-  const int64_t t = row - bh * g.N;
+  if (t >= (int)g.N) return;
+  const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
   const T* og = Og + bh * g.S * kD + c * 8;
+  const int S = (int)g.S;
   int32_t slot[L];
 #pragma unroll
   for (int l = 0; l < L; ++l) {
-    const int64_t i = ((t + 1) >> (g.logp * l)) - 1;
-    slot[l] = i >= 0 ? __ldg(inv + g.flat_off[l] + i) : -1;
-  }
-  float x[L][8];
-#pragma unroll
-  for (int l = 0; l < L; ++l) {
-    if (slot[l] >= 0 && slot[l] < g.S) Vec8<T>::load(og + (int64_t)slot[l] * kD, x[l]);
-    else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[l][e] = 0.f;
-    }
+    const int i = ((t + 1) >> (LOGP * l)) - 1;
+    slot[l] = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
   }
   float acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-    for (int l = 0; l < L; ++l) acc[e] += x[l][e];  // ascending level
+  for (int l = 0; l < L; ++l) {  // ascending level
+    if ((unsigned)slot[l] < (unsigned)S) {
+      float x[8];
+      Vec8<T>::load(og + (int64_t)slot[l] * kD, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += x[e];
+    }
   }
-  store_stream<T>(O + row * kD + c * 8, acc);
+  store_stream<T>(O + (bh * g.N + t) * kD + c * 8, acc);
 }
 
-template <typename T>
+template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
                    const int32_t* __restrict__ sel_idx, T* __restrict__ dOg, float* __restrict__ D) {
-  const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
+  const int j = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
   const int c = threadIdx.x & 7;
-  const bool live = row < g.BH * g.S;
-  const int64_t r = live ? row : 0;
-  const int64_t bh = r / g.S;
-  int64_t f = sel_idx[r];
-  if (f < 0 || f >= g.Ntot) f = g.Ntot - 1;  // unreachable for a valid selection
-  const int l = level_of(g, f);
-  const int64_t i = f - g.flat_off[l];
-  const int sh = g.logp * l;
-  const int64_t lo = ((i + 1) << sh) - 1;
-  const int64_t hi = min(lo + (int64_t(1) << sh) - 1, g.N - 1);
+  const int S = (int)g.S, N = (int)g.N;
+  const bool live = j < S;
+  const int64_t bh = blockIdx.y;
+  const int64_t r = bh * g.S + (live ? j : 0);
+  int f = sel_idx[r];
+  if (f < 0 || f >= (int)g.Ntot) f = (int)g.Ntot - 1;  // unreachable for a valid selection
+  int l = 0;
+#pragma unroll
+  for (int q = 1; q < L; ++q)
+    if (f >= (int)g.flat_off[q]) l = q;
+  const int i = f - (int)g.flat_off[l];
+  const int sh = LOGP * l;
+  const int lo = ((i + 1) << sh) - 1;
+  const int hi = min(lo + (1 << sh) - 1, N - 1);
   const T* src = dO + bh * g.N * kD + c * 8;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  for (int64_t t = lo; t <= hi; ++t) {
+  int t = lo;
+  for (; t + 3 <= hi; t += 4) {  // four independent row loads in flight
+    float x0[8], x1[8], x2[8], x3[8];
+    Vec8<T>::load(src + (int64_t)t * kD, x0);
+    Vec8<T>::load(src + (int64_t)(t + 1) * kD, x1);
+    Vec8<T>::load(src + (int64_t)(t + 2) * kD, x2);
+    Vec8<T>::load(src + (int64_t)(t + 3) * kD, x3);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += ((x0[e] + x1[e]) + (x2[e] + x3[e]));
+  }
+  for (; t <= hi; ++t) {
     float x[8];
-    Vec8<T>::load(src + t * kD, x);
+    Vec8<T>::load(src + (int64_t)t * kD, x);
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += x[e];
   }
@@ -162,43 +173,40 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   if (c == 0) D[r] = dsum;
 }
 
-template <typename T, int L>
+template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
                   T* __restrict__ dQ, T* __restrict__ dK, T* __restrict__ dV) {
-  const int64_t row = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
+  const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
   const int c = threadIdx.x & 7;
-  if (row >= g.BH * g.N) return;
-  const int64_t bh = row / g.N;
-  const int64_t t = row - bh * g.N;
+  if (t >= (int)g.N) return;
+  const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
   const int64_t base = bh * g.S * kD + c * 8;
+  const int S = (int)g.S;
   int32_t slot[L];
 #pragma unroll
-  for (int l = 0; l < L; ++l) slot[l] = __ldg(inv + g.flat_off[l] + (t >> (g.logp * l)));
+  for (int l = 0; l < L; ++l) slot[l] = __ldg(inv + (int)g.flat_off[l] + (t >> (LOGP * l)));
+  const int64_t out = (bh * g.N + t) * kD + c * 8;
   const T* src[3] = {dQg, dKg, dVg};
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
-    float x[L][8];
-#pragma unroll
-    for (int l = 0; l < L; ++l) {
-      if (slot[l] >= 0 && slot[l] < g.S) Vec8<T>::load(src[w] + base + (int64_t)slot[l] * kD, x[l]);
-      else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[l][e] = 0.f;
-      }
-    }
     float acc[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-      for (int l = 0; l < L; ++l)  // ascending level; 1/p^l is a power of two: exact
-        acc[e] = fmaf(x[l][e], 1.f / (float)(1 << (g.logp * l)), acc[e]);
+    for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
+      if ((unsigned)slot[l] < (unsigned)S) {
+        float x[8];
+        Vec8<T>::load(src[w] + base + (int64_t)slot[l] * kD, x);
+        const float wgt = 1.f / (float)(1 << (LOGP * l));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(x[e], wgt, acc[e]);
+      }
     }
-    store_stream<T>(dst[w] + row * kD + c * 8, acc);
+    store_stream<T>(dst[w] + out, acc);
   }
 }
 
@@ -225,71 +233,78 @@ cudaError_t launch_gather(const lh_plan& plan, const void* Q, const void* K, con
   return cudaGetLastError();
 }
 
-template <typename T, int L>
-void scatter_l(const Geo& g, unsigned b, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
-  scatter_kernel<T, L><<<b, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+// Calls f.template operator()<LOGP, L>() for the plan's p in {2, 4} and L <= 5.
+template <typename F>
+void with_levels(const Geo& g, F&& f) {
+  if (g.logp == 1) {
+    switch (g.L) {
+      case 1: f.template operator()<1, 1>(); break;
+      case 2: f.template operator()<1, 2>(); break;
+      case 3: f.template operator()<1, 3>(); break;
+      case 4: f.template operator()<1, 4>(); break;
+      default: f.template operator()<1, 5>(); break;
+    }
+  } else {
+    switch (g.L) {
+      case 1: f.template operator()<2, 1>(); break;
+      case 2: f.template operator()<2, 2>(); break;
+      case 3: f.template operator()<2, 3>(); break;
+      case 4: f.template operator()<2, 4>(); break;
+      default: f.template operator()<2, 5>(); break;
+    }
+  }
 }
 
 template <typename T>
-void scatter_t(const Geo& g, unsigned b, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
-  switch (g.L) {
-    case 1: scatter_l<T, 1>(g, b, Og, slot_of, O, st); break;
-    case 2: scatter_l<T, 2>(g, b, Og, slot_of, O, st); break;
-    case 3: scatter_l<T, 3>(g, b, Og, slot_of, O, st); break;
-    case 4: scatter_l<T, 4>(g, b, Og, slot_of, O, st); break;
-    default: scatter_l<T, 5>(g, b, Og, slot_of, O, st); break;
-  }
+void scatter_t(const Geo& g, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
+  const dim3 grid((unsigned)((g.N + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  with_levels(g, [&]<int LOGP, int L>() {
+    scatter_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+  });
 }
 
 cudaError_t launch_scatter(const lh_plan& plan, const void* Og, const int32_t* slot_of, void* O,
                            cudaStream_t st) {
   const Geo g = make_geo(plan);
-  const unsigned b = blocks_for(g.BH * g.N);
-  if (plan.c.dtype == LH_BF16) scatter_t<__nv_bfloat16>(g, b, Og, slot_of, O, st);
-  else scatter_t<float>(g, b, Og, slot_of, O, st);
+  if (plan.c.dtype == LH_BF16) scatter_t<__nv_bfloat16>(g, Og, slot_of, O, st);
+  else scatter_t<float>(g, Og, slot_of, O, st);
   return cudaGetLastError();
+}
+
+template <typename T>
+void scatter_bwd_t(const Geo& g, const void* dO, const void* Og, const int32_t* sel_idx, void* dOg,
+                   float* D, cudaStream_t st) {
+  const dim3 grid((unsigned)((g.S + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  with_levels(g, [&]<int LOGP, int L>() {
+    scatter_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og, sel_idx,
+                                                              (T*)dOg, D);
+  });
 }
 
 cudaError_t launch_scatter_bwd(const lh_plan& plan, const void* dO, const void* Og,
                                const int32_t* sel_idx, void* dOg, float* D, cudaStream_t st) {
   const Geo g = make_geo(plan);
-  const unsigned b = blocks_for(g.BH * g.S);
-  if (plan.c.dtype == LH_BF16) {
-    using T = __nv_bfloat16;
-    scatter_bwd_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og, sel_idx, (T*)dOg, D);
-  } else {
-    using T = float;
-    scatter_bwd_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og, sel_idx, (T*)dOg, D);
-  }
+  if (plan.c.dtype == LH_BF16) scatter_bwd_t<__nv_bfloat16>(g, dO, Og, sel_idx, dOg, D, st);
+  else scatter_bwd_t<float>(g, dO, Og, sel_idx, dOg, D, st);
   return cudaGetLastError();
 }
 
-template <typename T, int L>
-void gather_bwd_l(const Geo& g, unsigned b, const void* dQg, const void* dKg, const void* dVg,
-                  const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
-  gather_bwd_kernel<T, L><<<b, kThreads, 0, st>>>(g, (const T*)dQg, (const T*)dKg, (const T*)dVg,
-                                                  slot_of, (T*)dQ, (T*)dK, (T*)dV);
-}
-
 template <typename T>
-void gather_bwd_t(const Geo& g, unsigned b, const void* dQg, const void* dKg, const void* dVg,
+void gather_bwd_t(const Geo& g, const void* dQg, const void* dKg, const void* dVg,
                   const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
-  switch (g.L) {
-    case 1: gather_bwd_l<T, 1>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
-    case 2: gather_bwd_l<T, 2>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
-    case 3: gather_bwd_l<T, 3>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
-    case 4: gather_bwd_l<T, 4>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
-    default: gather_bwd_l<T, 5>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st); break;
-  }
+  const dim3 grid((unsigned)((g.N + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  with_levels(g, [&]<int LOGP, int L>() {
+    gather_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(
+        g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
+  });
 }
 
 cudaError_t launch_gather_bwd(const lh_plan& plan, const void* dQg, const void* dKg,
                               const void* dVg, const int32_t* slot_of, void* dQ, void* dK,
                               void* dV, cudaStream_t st) {
   const Geo g = make_geo(plan);
-  const unsigned b = blocks_for(g.BH * g.N);
-  if (plan.c.dtype == LH_BF16) gather_bwd_t<__nv_bfloat16>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
-  else gather_bwd_t<float>(g, b, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
+  if (plan.c.dtype == LH_BF16) gather_bwd_t<__nv_bfloat16>(g, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
+  else gather_bwd_t<float>(g, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
   return cudaGetLastError();
 }
 
