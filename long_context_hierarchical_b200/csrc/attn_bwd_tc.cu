@@ -6,22 +6,24 @@
 // dS = P (dP - D), D = rowsum(dO O):
 //   dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d).
 // Two kernels, deterministic, no atomics:
-//  - dk/dv: one CTA per 128-key tile walks the query tiles from its diagonal
-//    on.  S^T = K Q^T and dP^T = V dO^T land in TMEM (lane = key); the
-//    softmax warps turn them into P^T and dS^T (bf16, swizzled K-major smem);
-//    dV += P^T dO and dK += dS^T Q accumulate in TMEM.
-//  - dq: one CTA per 128-query tile walks the key tiles up to its diagonal.
-//    S = Q K^T and dP = dO V^T in TMEM (lane = query), dS to smem,
+//  - dk/dv: one CTA per 128-key tile streams query chunks of C rows from its
+//    diagonal on.  S^T = K Q^T and dP^T = V dO^T land in TMEM (lane = key);
+//    the element-wise warps turn them into P^T and dS^T (bf16, swizzled
+//    K-major smem); dV += P^T dO and dK += dS^T Q accumulate in TMEM.
+//  - dq: one CTA per 128-query tile streams key chunks of C rows up to its
+//    diagonal.  S = Q K^T and dP = dO V^T in TMEM (lane = query), dS to smem,
 //    dQ += dS K in TMEM.
-// Warp roles (576 threads): warps 0-15 are four element-wise groups of four
-// warps that split the 128 columns of each tile in quarters (no row
-// reductions are needed here), warp 16 loads (TMA for tiles, plain loads for
-// LSE/D), warp 17 owns TMEM and issues the MMAs from one thread.  TMEM columns: [0,128) S or
-// S^T, [128,256) dP or dP^T, [256,320) dQ or dV, [320,384) dK.
-// Overlap: each element-wise thread copies its S/dP columns out of TMEM and
-// releases them at once, so the next tile's S and dP MMAs run while it
-// computes; the single P/dS shared-memory tile has its own "consumed"
-// barrier that the element-wise warps wait on just before overwriting it.
+// Warp roles: C/32 element-wise groups of four warps split each step's C
+// columns (no row reductions are needed here), then one load warp (TMA for
+// tiles, plain loads for LSE/D) and one warp that owns TMEM and issues the
+// MMAs from one thread.  With C = 64 the TMEM (<= 256 columns) and shared
+// memory of a CTA fit twice on an SM, so two independent CTAs interleave
+// their MMA / element-wise / load latencies.
+// Overlap inside a CTA: each element-wise thread copies its S/dP columns out
+// of TMEM and releases them at once, so the next step's S and dP MMAs run
+// while it computes; the single P/dS shared-memory tile has its own
+// "consumed" barrier that the element-wise warps wait on just before
+// overwriting it.
 // Operand layouts are those of the forward kernel: K-major A/B tiles with the
 // 128-byte swizzle, tiles read as the MN-major B operand (dO, Q, K) with
 // 8-row groups 1024 bytes apart.  Every wait is bounded (see tc.cuh).
@@ -30,23 +32,34 @@
 
 namespace lh {
 
-bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows);
+bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows);
 
 namespace {
 
 using bf16 = __nv_bfloat16;
 using namespace tc;
 
-constexpr int kRows = 128;
-constexpr int kStages = 3;
-constexpr uint32_t kTile = kRows * kD * 2;      // 16 KB
-constexpr uint32_t kKBlock = kRows * 128;       // one 64-column K-block of a 128-wide tile
-constexpr uint32_t kWide = 2 * kKBlock;         // 32 KB: 128 x 128 bf16
-constexpr int kGroups = 4;                      // element-wise warp groups
-constexpr int kEw = kGroups * 128;              // element-wise threads
-constexpr int kLoadWarp = 4 * kGroups, kMmaWarp = kLoadWarp + 1;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
+constexpr int kRows = 128;                   // resident tile rows = MMA M
+constexpr uint32_t kTileR = kRows * kD * 2;  // 16 KB
+constexpr uint32_t kKBlock = kRows * 128;    // one 64-column K-block of a 128-row tile
 constexpr float kLog2e = 1.4426950408889634f;
+
+constexpr uint32_t pow2_cols(uint32_t n) {
+  return n <= 32 ? 32 : n <= 64 ? 64 : n <= 128 ? 128 : n <= 256 ? 256 : 512;
+}
+
+template <int C>
+struct Cfg {
+  static_assert(C == 64 || C == 128, "step width");
+  static constexpr int kGroups = C / 32;        // element-wise warp groups
+  static constexpr int kEw = kGroups * 128;     // element-wise threads
+  static constexpr int kLoadWarp = 4 * kGroups, kMmaWarp = kLoadWarp + 1;
+  static constexpr int kThreads = (kMmaWarp + 1) * 32;
+  static constexpr int kCtas = C == 64 ? 2 : 1;  // CTAs per SM
+  static constexpr int kStages = C == 64 ? 2 : 3;
+  static constexpr uint32_t kTileC = C * kD * 2;         // streamed tile bytes
+  static constexpr uint32_t kWide = (C / 64) * kKBlock;  // 128 x C bf16, K-major
+};
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -61,19 +74,17 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t* w) {
                : "memory");
 }
 
-// Row r of a 128 x 128 bf16 tile in the swizzled K-major layout: 16-byte
-// chunk ch (0..15) of the row.
-__device__ __forceinline__ uint32_t wide_chunk(uint32_t tile, int r, int ch) {
-  return tile + (ch >> 3) * kKBlock + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
-}
-
-// Writes columns [32 c0, 32 c0 + 32) of this thread's rows as bf16.
+// Writes columns [32 c0, 32 c0 + 32) of row r of a 128-row, swizzled K-major
+// tile (16-byte chunk ch of a row sits in K-block ch / 8).
 __device__ __forceinline__ void store_row32(uint32_t tile, int r, int c0, const uint32_t (&w)[16]) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) st_shared_v4(wide_chunk(tile, r, 4 * c0 + q), &w[4 * q]);
+  for (int q = 0; q < 4; ++q) {
+    const int ch = 4 * c0 + q;
+    st_shared_v4(tile + (ch >> 3) * kKBlock + r * 128 + (((ch & 7) ^ (r & 7)) << 4), &w[4 * q]);
+  }
 }
 
-// 64 columns of a TMEM lane as one bf16 row (scaled) into global memory.
+// 32 fp32 values of a TMEM lane as bf16 (scaled) into global memory.
 __device__ __forceinline__ void store_out32(bf16* dst, const float (&v)[32], float scale) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -84,176 +95,186 @@ __device__ __forceinline__ void store_out32(bf16* dst, const float (&v)[32], flo
   }
 }
 
+// D[tmem] = A(128 x 64, K-major tile) * B(N x 64, K-major tile)^T.  Descriptors
+// are built once per tile and advanced by adds: the issuing thread is serial.
+__device__ __forceinline__ void gemm_sq(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc) {
+  const uint64_t da = sw128_desc(a, 16, 1024), db = sw128_desc(b, 16, 1024);
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) mma_bf16(d, desc_add(da, ks * 32), desc_add(db, ks * 32), idesc, ks > 0);
+}
+// D[tmem] (+)= A(128 x C, K-major wide tile) * B(C x 64 tile read MN-major)
+template <int C>
+__device__ __forceinline__ void gemm_acc(uint32_t d, uint32_t a, uint32_t b, bool acc) {
+  constexpr uint32_t idesc = idesc_bf16(kRows, kD, true);
+  const uint64_t da = sw128_desc(a, 16, 1024), db = sw128_desc(b, Cfg<C>::kTileC, 1024);
+#pragma unroll
+  for (int kk = 0; kk < C / 16; ++kk)
+    mma_bf16(d, desc_add(da, (kk >> 2) * kKBlock + (kk & 3) * 32), desc_add(db, kk * 2048), idesc,
+             (acc || kk > 0) ? 1u : 0u);
+}
+
 // ===========================================================================
 // dK, dV
 // ===========================================================================
-namespace kv {
-constexpr uint32_t kOffK = 0, kOffV = kTile;
-constexpr uint32_t kOffQ = 2 * kTile;                    // kStages tiles
-constexpr uint32_t kOffG = kOffQ + kStages * kTile;      // dO, kStages tiles
-constexpr uint32_t kOffPT = kOffG + kStages * kTile;     // P^T  (128 x 128)
-constexpr uint32_t kOffDST = kOffPT + kWide;             // dS^T (128 x 128)
-constexpr uint32_t kOffVec = kOffDST + kWide;            // kStages x (128 lse2 + 128 D) fp32
-constexpr uint32_t kOffBar = kOffVec + kStages * 1024;
-constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * kStages,
-                   kBarSP = kBarEmpty + 8 * kStages, kBarPDS = kBarSP + 8, kBarAcc = kBarPDS + 8,
-                   kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8, kBarPF = kBarTF + 8,
-                   kSlotTmem = kBarPF + 8, kSlotAbort = kSlotTmem + 4;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-}  // namespace kv
+template <int C>
+struct KV {
+  using F = Cfg<C>;
+  static constexpr uint32_t kOffK = 0, kOffV = kTileR;
+  static constexpr uint32_t kOffQ = 2 * kTileR;                       // kStages tiles
+  static constexpr uint32_t kOffG = kOffQ + F::kStages * F::kTileC;   // dO, kStages tiles
+  static constexpr uint32_t kOffPT = kOffG + F::kStages * F::kTileC;  // P^T  (128 x C)
+  static constexpr uint32_t kOffDST = kOffPT + F::kWide;              // dS^T (128 x C)
+  static constexpr uint32_t kOffVec = kOffDST + F::kWide;             // kStages x (C lse2 + C D)
+  static constexpr uint32_t kOffBar = kOffVec + F::kStages * 2 * C * 4;
+  static constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * F::kStages,
+                            kBarSP = kBarEmpty + 8 * F::kStages, kBarPDS = kBarSP + 8,
+                            kBarAcc = kBarPDS + 8, kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8,
+                            kBarPF = kBarTF + 8, kSlotTmem = kBarPF + 8, kSlotAbort = kSlotTmem + 4;
+  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr uint32_t kTmemCols = pow2_cols(2 * C + 2 * kD);
+};
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int C>
+__global__ void __launch_bounds__(Cfg<C>::kThreads, Cfg<C>::kCtas)
 attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                         const float* __restrict__ lse, const float* __restrict__ Dv,
-                        bf16* __restrict__ dK, bf16* __restrict__ dV, int S, int ntiles, float sl2,
-                        float scale, unsigned int* __restrict__ status) {
-  using namespace kv;
+                        bf16* __restrict__ dK, bf16* __restrict__ dV, int S, float sl2, float scale,
+                        unsigned int* __restrict__ status) {
+  using F = Cfg<C>;
+  using L = KV<C>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t bars = base + kOffBar;
-  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + kSlotAbort);
-  const float* vec = reinterpret_cast<const float*>(gbase + kOffVec);
+  const uint32_t bars = base + L::kOffBar;
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + L::kOffBar + L::kSlotAbort);
+  const float* vec = reinterpret_cast<const float*>(gbase + L::kOffVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // key tile; tile 0 sees the most query tiles
+  const int kt = blockIdx.x;  // key tile; tile 0 sees the most query chunks
   const int bh = blockIdx.y;
   const int k0 = kt * kRows;
-  const int nq = ntiles - kt;  // query tiles kt .. ntiles-1
+  const int nq = (S - k0 + C - 1) / C;  // query chunks [k0 + C t, k0 + C t + C)
   const int row0 = bh * S;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + kBarKV, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + kBarFull + 8 * s, 33);  // TMA (expect_tx) + 32 vector lanes
-      mbar_init(bars + kBarEmpty + 8 * s, 1);
+    mbar_init(bars + L::kBarKV, 1);
+    for (int s = 0; s < F::kStages; ++s) {
+      mbar_init(bars + L::kBarFull + 8 * s, 33);  // TMA (expect_tx) + 32 vector lanes
+      mbar_init(bars + L::kBarEmpty + 8 * s, 1);
     }
-    mbar_init(bars + kBarSP, 1);
-    mbar_init(bars + kBarPDS, kEw);
-    mbar_init(bars + kBarAcc, 1);
-    mbar_init(bars + kBarDrain, 1);
-    mbar_init(bars + kBarTF, kEw);  // S^T/dP^T copied out of TMEM
-    mbar_init(bars + kBarPF, 1);    // P^T/dS^T tile consumed by the MMAs
+    mbar_init(bars + L::kBarSP, 1);
+    mbar_init(bars + L::kBarPDS, F::kEw);
+    mbar_init(bars + L::kBarAcc, 1);
+    mbar_init(bars + L::kBarDrain, 1);
+    mbar_init(bars + L::kBarTF, F::kEw);  // S^T/dP^T copied out of TMEM
+    mbar_init(bars + L::kBarPF, 1);       // P^T/dS^T tile consumed by the MMAs
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) tmem_alloc(bars + kSlotTmem, 512);
+  if (warp == F::kMmaWarp) tmem_alloc(bars + L::kSlotTmem, L::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kOffBar + L::kSlotTmem);
 
-  if (warp == kLoadWarp) {
+  if (warp == F::kLoadWarp) {
     // ---------------- loads ----------------
     int issued = 0;
     if (lane == 0) {
-      mbar_expect_tx(bars + kBarKV, 2 * kTile);
-      tma_load_2d(base + kOffK, &tmK, 0, row0 + k0, bars + kBarKV);
-      tma_load_2d(base + kOffV, &tmV, 0, row0 + k0, bars + kBarKV);
+      mbar_expect_tx(bars + L::kBarKV, 2 * kTileR);
+      tma_load_2d(base + L::kOffK, &tmK, 0, row0 + k0, bars + L::kBarKV);
+      tma_load_2d(base + L::kOffV, &tmV, 0, row0 + k0, bars + L::kBarKV);
     }
     for (int t = 0; t < nq; ++t) {
-      const int s = t % kStages, u = t / kStages;
+      const int s = t % F::kStages, u = t / F::kStages;
       bool go = true;
-      if (t >= kStages) go = mbar_wait(bars + kBarEmpty + 8 * s, (u - 1) & 1, abort, status);
+      if (t >= F::kStages) go = mbar_wait(bars + L::kBarEmpty + 8 * s, (u - 1) & 1, abort, status);
       if (!__all_sync(0xffffffffu, go)) break;
-      const int q0 = (kt + t) * kRows;
+      const int q0 = k0 + t * C;
       if (lane == 0) {
-        mbar_expect_tx(bars + kBarFull + 8 * s, 2 * kTile);
-        tma_load_2d(base + kOffQ + s * kTile, &tmQ, 0, row0 + q0, bars + kBarFull + 8 * s);
-        tma_load_2d(base + kOffG + s * kTile, &tmG, 0, row0 + q0, bars + kBarFull + 8 * s);
+        mbar_expect_tx(bars + L::kBarFull + 8 * s, 2 * F::kTileC);
+        tma_load_2d(base + L::kOffQ + s * F::kTileC, &tmQ, 0, row0 + q0, bars + L::kBarFull + 8 * s);
+        tma_load_2d(base + L::kOffG + s * F::kTileC, &tmG, 0, row0 + q0, bars + L::kBarFull + 8 * s);
       }
-      float* dst = reinterpret_cast<float*>(gbase + kOffVec + s * 1024);
+      float* dst = reinterpret_cast<float*>(gbase + L::kOffVec + s * 2 * C * 4);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < C / 32; ++e) {
         const int q = 32 * e + lane;
         const bool in = q0 + q < S;
         dst[q] = in ? lse[row0 + q0 + q] * kLog2e : 0.f;
-        dst[128 + q] = in ? Dv[row0 + q0 + q] : 0.f;
+        dst[C + q] = in ? Dv[row0 + q0 + q] : 0.f;
       }
-      mbar_arrive(bars + kBarFull + 8 * s);
+      mbar_arrive(bars + L::kBarFull + 8 * s);
       issued = t + 1;
     }
     if (lane == 0 && *abort) {
-      wait_drain(bars + kBarKV, 0);
-      for (int t = issued - kStages < 0 ? 0 : issued - kStages; t < issued; ++t)
-        wait_drain(bars + kBarFull + 8 * (t % kStages), (t / kStages) & 1);
+      wait_drain(bars + L::kBarKV, 0);
+      for (int t = issued - F::kStages < 0 ? 0 : issued - F::kStages; t < issued; ++t)
+        wait_drain(bars + L::kBarFull + 8 * (t % F::kStages), (t / F::kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == F::kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idSq = idesc_bf16(kRows, kRows, false);
-      constexpr uint32_t idAcc = idesc_bf16(kRows, kD, true);
-      // D[tmem] = A(128 x 64, K-major tile) * B(128 x 64, K-major tile)^T
-      auto gemm_sq = [&](uint32_t d, uint32_t a, uint32_t b) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16(d, sw128_desc(a + ks * 32, 16, 1024), sw128_desc(b + ks * 32, 16, 1024), idSq, ks > 0);
-      };
-      // D[tmem] (+)= A(128 x 128, K-major wide tile) * B(128 x 64 tile, MN-major)
-      auto gemm_acc = [&](uint32_t d, uint32_t a, uint32_t b, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(d, sw128_desc(a + (kk >> 2) * kKBlock + (kk & 3) * 32, 16, 1024),
-                   sw128_desc(b + kk * 2048, kTile, 1024), idAcc, (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(bars + kBarKV, 0, abort, status) && mbar_wait(bars + kBarFull, 0, abort, status);
+      constexpr uint32_t idS = idesc_bf16(kRows, C, false);
+      bool ok = mbar_wait(bars + L::kBarKV, 0, abort, status) &&
+                mbar_wait(bars + L::kBarFull, 0, abort, status);
       if (ok) {
         tc_fence_after();
-        gemm_sq(tmem, base + kOffK, base + kOffQ);                // S^T = K Q^T
-        gemm_sq(tmem + kRows, base + kOffV, base + kOffG);        // dP^T = V dO^T
-        mma_commit(bars + kBarSP);
+        gemm_sq(tmem, base + L::kOffK, base + L::kOffQ, idS);      // S^T = K Q^T
+        gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG, idS);  // dP^T = V dO^T
+        mma_commit(bars + L::kBarSP);
       }
       for (int t = 0; ok && t < nq; ++t) {
-        const int s = t % kStages;
-        // S^T/dP^T of tile t copied out: start tile t+1's while tile t computes
-        if (!(ok = mbar_wait(bars + kBarTF, t & 1, abort, status))) break;
+        const int s = t % F::kStages;
+        // S^T/dP^T of step t copied out: start step t+1's while step t computes
+        if (!(ok = mbar_wait(bars + L::kBarTF, t & 1, abort, status))) break;
         tc_fence_after();
         if (t + 1 < nq) {
-          const int s1 = (t + 1) % kStages, u1 = (t + 1) / kStages;
-          if (!(ok = mbar_wait(bars + kBarFull + 8 * s1, u1 & 1, abort, status))) break;
-          gemm_sq(tmem, base + kOffK, base + kOffQ + s1 * kTile);
-          gemm_sq(tmem + kRows, base + kOffV, base + kOffG + s1 * kTile);
-          mma_commit(bars + kBarSP);
+          const int s1 = (t + 1) % F::kStages, u1 = (t + 1) / F::kStages;
+          if (!(ok = mbar_wait(bars + L::kBarFull + 8 * s1, u1 & 1, abort, status))) break;
+          gemm_sq(tmem, base + L::kOffK, base + L::kOffQ + s1 * F::kTileC, idS);
+          gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG + s1 * F::kTileC, idS);
+          mma_commit(bars + L::kBarSP);
         }
-        if (!(ok = mbar_wait(bars + kBarPDS, t & 1, abort, status))) break;
+        if (!(ok = mbar_wait(bars + L::kBarPDS, t & 1, abort, status))) break;
         tc_fence_after();
-        gemm_acc(tmem + 2 * kRows, base + kOffPT, base + kOffG + s * kTile, t > 0);       // dV += P^T dO
-        gemm_acc(tmem + 2 * kRows + kD, base + kOffDST, base + kOffQ + s * kTile, t > 0); // dK += dS^T Q
-        mma_commit(bars + kBarPF);
-        mma_commit(bars + kBarEmpty + 8 * s);
+        gemm_acc<C>(tmem + 2 * C, base + L::kOffPT, base + L::kOffG + s * F::kTileC, t > 0);       // dV += P^T dO
+        gemm_acc<C>(tmem + 2 * C + kD, base + L::kOffDST, base + L::kOffQ + s * F::kTileC, t > 0); // dK += dS^T Q
+        mma_commit(bars + L::kBarPF);
+        mma_commit(bars + L::kBarEmpty + 8 * s);
       }
-      if (ok) mma_commit(bars + kBarAcc);
-      mma_commit(bars + kBarDrain);
-      wait_drain(bars + kBarDrain, 0);
+      if (ok) mma_commit(bars + L::kBarAcc);
+      mma_commit(bars + L::kBarDrain);
+      wait_drain(bars + L::kBarDrain, 0);
     }
   } else {
     // ---------------- element-wise: P^T, dS^T ----------------
     const int grp = warp >> 2, wr = warp & 3;
     const int r = wr * 32 + lane;  // key row of the tile = TMEM lane
     const int key = k0 + r;
-    const int col0 = grp * 32;     // this group's 32 query columns
+    const int col0 = grp * 32;     // this group's 32 query columns of the step
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
-      const int s = t % kStages;
-      ok = mbar_wait(bars + kBarSP, t & 1, abort, status);
-      if (ok) ok = mbar_wait(bars + kBarFull + 8 * s, (t / kStages) & 1, abort, status);
+      const int s = t % F::kStages;
+      ok = mbar_wait(bars + L::kBarSP, t & 1, abort, status);
+      if (ok) ok = mbar_wait(bars + L::kBarFull + 8 * s, (t / F::kStages) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const int q0 = (kt + t) * kRows;
+      const int q0 = k0 + t * C;
       // visible: key <= query < S
-      const bool edge = (t == 0) || (q0 + kRows > S);
-      const float* l2 = vec + s * 256 + col0;
-      const float* dd = l2 + 128;
+      const bool edge = (q0 < k0 + kRows) || (q0 + C > S);
+      const float* l2 = vec + s * 2 * C + col0;
+      const float* dd = l2 + C;
       float st[32], dp[32];
       tmem_ld32(lane_base + col0, st);
-      tmem_ld32(lane_base + kRows + col0, dp);
+      tmem_ld32(lane_base + C + col0, dp);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
+      mbar_arrive(bars + L::kBarTF);  // TMEM columns free for the next step's MMAs
       uint32_t wp[16], wd[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
@@ -274,184 +295,187 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         wd[e >> 1] = pack_bf16x2(p[0] * (dp[e] - dv.x), p[1] * (dp[e + 1] - dv.y));
         wd[(e >> 1) + 1] = pack_bf16x2(p[2] * (dp[e + 2] - dv.z), p[3] * (dp[e + 3] - dv.w));
       }
-      // the previous tile's P^T / dS^T must be consumed before they are overwritten
-      if (t > 0) ok = mbar_wait(bars + kBarPF, (t - 1) & 1, abort, status);
+      // the previous step's P^T / dS^T must be consumed before they are overwritten
+      if (t > 0) ok = mbar_wait(bars + L::kBarPF, (t - 1) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      store_row32(base + kOffPT, r, grp, wp);
-      store_row32(base + kOffDST, r, grp, wd);
+      store_row32(base + L::kOffPT, r, grp, wp);
+      store_row32(base + L::kOffDST, r, grp, wd);
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(bars + kBarPDS);
+      mbar_arrive(bars + L::kBarPDS);
     }
-    if (ok) ok = mbar_wait(bars + kBarAcc, 0, abort, status);
+    if (ok) ok = mbar_wait(bars + L::kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
-      // groups 0,1: dV columns [32 grp, +32); groups 2,3: dK columns [32 (grp-2), +32)
+      // TMEM [2C, 2C+64) = dV, [2C+64, 2C+128) = dK: 128 columns over the groups
       tc_fence_after();
-      const bool isk = grp >= 2;
-      const int c = (grp & 1) * 32;
-      float v[32];
-      tmem_ld32(lane_base + 2 * kRows + (isk ? kD : 0) + c, v);
-      tmem_wait_ld();
-      if (key < S)
-        store_out32((isk ? dK : dV) + ((int64_t)row0 + key) * kD + c, v, isk ? scale : 1.f);
+#pragma unroll
+      for (int piece = 0; piece < 4 / F::kGroups; ++piece) {
+        const int c = (grp * (4 / F::kGroups) + piece) * 32;  // 0..127
+        float v[32];
+        tmem_ld32(lane_base + 2 * C + c, v);
+        tmem_wait_ld();
+        if (key < S) {
+          const bool isk = c >= kD;
+          store_out32((isk ? dK : dV) + ((int64_t)row0 + key) * kD + (c & (kD - 1)), v,
+                      isk ? scale : 1.f);
+        }
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == F::kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
 
 // ===========================================================================
 // dQ
 // ===========================================================================
-namespace qq {
-constexpr uint32_t kOffQ = 0, kOffG = kTile;
-constexpr uint32_t kOffK = 2 * kTile;                  // kStages tiles
-constexpr uint32_t kOffV = kOffK + kStages * kTile;    // kStages tiles
-constexpr uint32_t kOffDS = kOffV + kStages * kTile;   // dS (128 x 128)
-constexpr uint32_t kOffBar = kOffDS + kWide;
-constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
-                   kBarSP = kBarE + 8 * kStages, kBarDS = kBarSP + 8, kBarAcc = kBarDS + 8,
-                   kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8, kBarDF = kBarTF + 8,
-                   kSlotTmem = kBarDF + 8, kSlotAbort = kSlotTmem + 4;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-}  // namespace qq
+template <int C>
+struct QQ {
+  using F = Cfg<C>;
+  static constexpr uint32_t kOffQ = 0, kOffG = kTileR;
+  static constexpr uint32_t kOffK = 2 * kTileR;                       // kStages tiles
+  static constexpr uint32_t kOffV = kOffK + F::kStages * F::kTileC;   // kStages tiles
+  static constexpr uint32_t kOffDS = kOffV + F::kStages * F::kTileC;  // dS (128 x C)
+  static constexpr uint32_t kOffBar = kOffDS + F::kWide;
+  static constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * F::kStages,
+                            kBarE = kBarV + 8 * F::kStages, kBarSP = kBarE + 8 * F::kStages,
+                            kBarDS = kBarSP + 8, kBarAcc = kBarDS + 8, kBarDrain = kBarAcc + 8,
+                            kBarTF = kBarDrain + 8, kBarDF = kBarTF + 8, kSlotTmem = kBarDF + 8,
+                            kSlotAbort = kSlotTmem + 4;
+  static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr uint32_t kTmemCols = pow2_cols(2 * C + kD);
+};
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int C>
+__global__ void __launch_bounds__(Cfg<C>::kThreads, Cfg<C>::kCtas)
 attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                       const float* __restrict__ lse, const float* __restrict__ Dv,
                       bf16* __restrict__ dQ, int S, int ntiles, float sl2, float scale,
                       unsigned int* __restrict__ status) {
-  using namespace qq;
+  using F = Cfg<C>;
+  using L = QQ<C>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t bars = base + kOffBar;
-  volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + kSlotAbort);
+  const uint32_t bars = base + L::kOffBar;
+  volatile int* abort = reinterpret_cast<volatile int*>(gbase + L::kOffBar + L::kSlotAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = ntiles - 1 - (int)blockIdx.x;  // longest rows first
   const int bh = blockIdx.y;
   const int q0 = qt * kRows;
-  const int nk = qt + 1;
+  const int kend = min(q0 + kRows, S);  // keys [0, kend) reach this tile
+  const int nk = (kend + C - 1) / C;
   const int row0 = bh * S;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars + kBarQ, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + kBarK + 8 * s, 1);
-      mbar_init(bars + kBarV + 8 * s, 1);
-      mbar_init(bars + kBarE + 8 * s, 1);
+    mbar_init(bars + L::kBarQ, 1);
+    for (int s = 0; s < F::kStages; ++s) {
+      mbar_init(bars + L::kBarK + 8 * s, 1);
+      mbar_init(bars + L::kBarV + 8 * s, 1);
+      mbar_init(bars + L::kBarE + 8 * s, 1);
     }
-    mbar_init(bars + kBarSP, 1);
-    mbar_init(bars + kBarDS, kEw);
-    mbar_init(bars + kBarAcc, 1);
-    mbar_init(bars + kBarDrain, 1);
-    mbar_init(bars + kBarTF, kEw);  // S/dP copied out of TMEM
-    mbar_init(bars + kBarDF, 1);    // dS tile consumed by the MMA
+    mbar_init(bars + L::kBarSP, 1);
+    mbar_init(bars + L::kBarDS, F::kEw);
+    mbar_init(bars + L::kBarAcc, 1);
+    mbar_init(bars + L::kBarDrain, 1);
+    mbar_init(bars + L::kBarTF, F::kEw);  // S/dP copied out of TMEM
+    mbar_init(bars + L::kBarDF, 1);       // dS tile consumed by the MMA
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) tmem_alloc(bars + kSlotTmem, 512);
+  if (warp == F::kMmaWarp) tmem_alloc(bars + L::kSlotTmem, L::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + kOffBar + kSlotTmem);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kOffBar + L::kSlotTmem);
 
-  if (warp == kLoadWarp) {
+  if (warp == F::kLoadWarp) {
     if (lane == 0) {
       int issued = 0;
-      mbar_expect_tx(bars + kBarQ, 2 * kTile);
-      tma_load_2d(base + kOffQ, &tmQ, 0, row0 + q0, bars + kBarQ);
-      tma_load_2d(base + kOffG, &tmG, 0, row0 + q0, bars + kBarQ);
+      mbar_expect_tx(bars + L::kBarQ, 2 * kTileR);
+      tma_load_2d(base + L::kOffQ, &tmQ, 0, row0 + q0, bars + L::kBarQ);
+      tma_load_2d(base + L::kOffG, &tmG, 0, row0 + q0, bars + L::kBarQ);
       for (int j = 0; j < nk; ++j) {
-        const int s = j % kStages, u = j / kStages;
-        if (j >= kStages && !mbar_wait(bars + kBarE + 8 * s, (u - 1) & 1, abort, status)) break;
-        mbar_expect_tx(bars + kBarK + 8 * s, kTile);
-        tma_load_2d(base + kOffK + s * kTile, &tmK, 0, row0 + j * kRows, bars + kBarK + 8 * s);
-        mbar_expect_tx(bars + kBarV + 8 * s, kTile);
-        tma_load_2d(base + kOffV + s * kTile, &tmV, 0, row0 + j * kRows, bars + kBarV + 8 * s);
+        const int s = j % F::kStages, u = j / F::kStages;
+        if (j >= F::kStages && !mbar_wait(bars + L::kBarE + 8 * s, (u - 1) & 1, abort, status)) break;
+        mbar_expect_tx(bars + L::kBarK + 8 * s, F::kTileC);
+        tma_load_2d(base + L::kOffK + s * F::kTileC, &tmK, 0, row0 + j * C, bars + L::kBarK + 8 * s);
+        mbar_expect_tx(bars + L::kBarV + 8 * s, F::kTileC);
+        tma_load_2d(base + L::kOffV + s * F::kTileC, &tmV, 0, row0 + j * C, bars + L::kBarV + 8 * s);
         issued = j + 1;
       }
       if (*abort) {
-        wait_drain(bars + kBarQ, 0);
-        for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j) {
-          wait_drain(bars + kBarK + 8 * (j % kStages), (j / kStages) & 1);
-          wait_drain(bars + kBarV + 8 * (j % kStages), (j / kStages) & 1);
+        wait_drain(bars + L::kBarQ, 0);
+        for (int j = issued - F::kStages < 0 ? 0 : issued - F::kStages; j < issued; ++j) {
+          wait_drain(bars + L::kBarK + 8 * (j % F::kStages), (j / F::kStages) & 1);
+          wait_drain(bars + L::kBarV + 8 * (j % F::kStages), (j / F::kStages) & 1);
         }
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == F::kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idSq = idesc_bf16(kRows, kRows, false);
-      constexpr uint32_t idAcc = idesc_bf16(kRows, kD, true);
-      auto gemm_sq = [&](uint32_t d, uint32_t a, uint32_t b) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_bf16(d, sw128_desc(a + ks * 32, 16, 1024), sw128_desc(b + ks * 32, 16, 1024), idSq, ks > 0);
-      };
-      bool ok = mbar_wait(bars + kBarQ, 0, abort, status) && mbar_wait(bars + kBarK, 0, abort, status) &&
-                mbar_wait(bars + kBarV, 0, abort, status);
+      constexpr uint32_t idS = idesc_bf16(kRows, C, false);
+      bool ok = mbar_wait(bars + L::kBarQ, 0, abort, status) && mbar_wait(bars + L::kBarK, 0, abort, status) &&
+                mbar_wait(bars + L::kBarV, 0, abort, status);
       if (ok) {
         tc_fence_after();
-        gemm_sq(tmem, base + kOffQ, base + kOffK);           // S = Q K^T
-        gemm_sq(tmem + kRows, base + kOffG, base + kOffV);   // dP = dO V^T
-        mma_commit(bars + kBarSP);
+        gemm_sq(tmem, base + L::kOffQ, base + L::kOffK, idS);      // S = Q K^T
+        gemm_sq(tmem + C, base + L::kOffG, base + L::kOffV, idS);  // dP = dO V^T
+        mma_commit(bars + L::kBarSP);
       }
       for (int j = 0; ok && j < nk; ++j) {
-        const int s = j % kStages;
-        if (!(ok = mbar_wait(bars + kBarTF, j & 1, abort, status))) break;
+        const int s = j % F::kStages;
+        if (!(ok = mbar_wait(bars + L::kBarTF, j & 1, abort, status))) break;
         tc_fence_after();
         if (j + 1 < nk) {
-          const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
-          if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
-          if (!(ok = mbar_wait(bars + kBarV + 8 * s1, u1 & 1, abort, status))) break;
-          gemm_sq(tmem, base + kOffQ, base + kOffK + s1 * kTile);
-          gemm_sq(tmem + kRows, base + kOffG, base + kOffV + s1 * kTile);
-          mma_commit(bars + kBarSP);
+          const int s1 = (j + 1) % F::kStages, u1 = (j + 1) / F::kStages;
+          if (!(ok = mbar_wait(bars + L::kBarK + 8 * s1, u1 & 1, abort, status))) break;
+          if (!(ok = mbar_wait(bars + L::kBarV + 8 * s1, u1 & 1, abort, status))) break;
+          gemm_sq(tmem, base + L::kOffQ, base + L::kOffK + s1 * F::kTileC, idS);
+          gemm_sq(tmem + C, base + L::kOffG, base + L::kOffV + s1 * F::kTileC, idS);
+          mma_commit(bars + L::kBarSP);
         }
-        if (!(ok = mbar_wait(bars + kBarDS, j & 1, abort, status))) break;
+        if (!(ok = mbar_wait(bars + L::kBarDS, j & 1, abort, status))) break;
         tc_fence_after();
-        const uint32_t kk_tile = base + kOffK + s * kTile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dQ += dS K
-          mma_bf16(tmem + 2 * kRows, sw128_desc(base + kOffDS + (kk >> 2) * kKBlock + (kk & 3) * 32, 16, 1024),
-                   sw128_desc(kk_tile + kk * 2048, kTile, 1024), idAcc, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bars + kBarDF);
-        mma_commit(bars + kBarE + 8 * s);
+        gemm_acc<C>(tmem + 2 * C, base + L::kOffDS, base + L::kOffK + s * F::kTileC, j > 0);  // dQ += dS K
+        mma_commit(bars + L::kBarDF);
+        mma_commit(bars + L::kBarE + 8 * s);
       }
-      if (ok) mma_commit(bars + kBarAcc);
-      mma_commit(bars + kBarDrain);
-      wait_drain(bars + kBarDrain, 0);
+      if (ok) mma_commit(bars + L::kBarAcc);
+      mma_commit(bars + L::kBarDrain);
+      wait_drain(bars + L::kBarDrain, 0);
     }
   } else {
     const int grp = warp >> 2, wr = warp & 3;
     const int r = wr * 32 + lane;
     const int qrow = q0 + r;
-    const int col0 = grp * 32;  // this group's 32 key columns
+    const int col0 = grp * 32;  // this group's 32 key columns of the step
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
     const float l2 = qrow < S ? lse[row0 + qrow] * kLog2e : 0.f;
     const float Dr = qrow < S ? Dv[row0 + qrow] : 0.f;
     const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-l2, -l2);
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
-      ok = mbar_wait(bars + kBarSP, j & 1, abort, status);
+      ok = mbar_wait(bars + L::kBarSP, j & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      const bool diag = j == nk - 1;
-      const int lim = qrow - j * kRows - col0;  // visible columns of this group: c <= lim
+      const int kc = j * C + col0;     // first key of this group's columns
+      const bool diag = kc + 31 > q0;  // some key may follow some query of the tile
+      const int lim = qrow - kc;       // visible columns: e <= lim
       float sv[32], dp[32];
       tmem_ld32(lane_base + col0, sv);
-      tmem_ld32(lane_base + kRows + col0, dp);
+      tmem_ld32(lane_base + C + col0, dp);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bars + kBarTF);  // TMEM columns free for the next tile's MMAs
+      mbar_arrive(bars + L::kBarTF);  // TMEM columns free for the next step's MMAs
       uint32_t w[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
@@ -463,18 +487,18 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         }
         w[e >> 1] = pack_bf16x2(pa * (dp[e] - Dr), pb * (dp[e + 1] - Dr));
       }
-      if (j > 0) ok = mbar_wait(bars + kBarDF, (j - 1) & 1, abort, status);
+      if (j > 0) ok = mbar_wait(bars + L::kBarDF, (j - 1) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      store_row32(base + kOffDS, r, grp, w);
+      store_row32(base + L::kOffDS, r, grp, w);
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(bars + kBarDS);
+      mbar_arrive(bars + L::kBarDS);
     }
-    if (ok) ok = mbar_wait(bars + kBarAcc, 0, abort, status);
+    if (ok) ok = mbar_wait(bars + L::kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok) && grp < 2) {
       tc_fence_after();
       float v[32];
-      tmem_ld32(lane_base + 2 * kRows + grp * 32, v);
+      tmem_ld32(lane_base + 2 * C + grp * 32, v);
       tmem_wait_ld();
       if (qrow < S) store_out32(dQ + ((int64_t)row0 + qrow) * kD + grp * 32, v, scale);
     }
@@ -482,42 +506,50 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == F::kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, L::kTmemCols);
   }
 }
+
+constexpr int kStep = 64;  // streamed rows per step
 
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                const float* lse, const void* dO, const float* D, void* dQ,
                                void* dK, void* dV, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mg;
-  if (!make_tile_map(&mq, Q, BH * S) || !make_tile_map(&mk, K, BH * S) ||
-      !make_tile_map(&mv, V, BH * S) || !make_tile_map(&mg, dO, BH * S))
+  constexpr int C = kStep;
+  using F = Cfg<C>;
+  // Tiles that stay resident in a CTA have 128 rows; streamed chunks have C.
+  CUtensorMap qR, gR, kR, vR, qC, gC, kC, vC;
+  const int64_t rows = BH * S;
+  if (!make_tile_map(&qR, Q, rows, kRows) || !make_tile_map(&gR, dO, rows, kRows) ||
+      !make_tile_map(&kR, K, rows, kRows) || !make_tile_map(&vR, V, rows, kRows) ||
+      !make_tile_map(&qC, Q, rows, C) || !make_tile_map(&gC, dO, rows, C) ||
+      !make_tile_map(&kC, K, rows, C) || !make_tile_map(&vC, V, rows, C))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kv::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<C>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, KV<C>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             qq::kSmemBytes);
+    e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QQ<C>::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float sl2 = 0.125f * kLog2e;
   const dim3 grid(ntiles, (unsigned)BH);
-  attn_bwd_dkdv_tc_kernel<<<grid, kThreads, kv::kSmemBytes, st>>>(
-      mq, mk, mv, mg, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, ntiles, sl2,
-      0.125f, status);
+  attn_bwd_dkdv_tc_kernel<C><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
+      qC, kR, vR, gC, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2, 0.125f,
+      status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_tc_kernel<<<grid, kThreads, qq::kSmemBytes, st>>>(
-      mq, mk, mv, mg, lse, D, static_cast<bf16*>(dQ), (int)S, ntiles, sl2, 0.125f, status);
+  attn_bwd_dq_tc_kernel<C><<<grid, F::kThreads, QQ<C>::kSmemBytes, st>>>(
+      qR, kC, vC, gR, lse, D, static_cast<bf16*>(dQ), (int)S, ntiles, sl2, 0.125f, status);
   return cudaGetLastError();
 }
 

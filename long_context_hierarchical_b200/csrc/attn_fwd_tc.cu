@@ -140,20 +140,22 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kRows, kRows, false);
       constexpr uint32_t idPV = idesc_bf16(kRows, kD, true);
+      // Descriptors are built once per tile and advanced by adds: this
+      // thread issues every MMA of the CTA.
       auto issue_S = [&](int x, int j) {
-        const uint32_t q = base + kOffQ + x * kTile, k = base + kOffK + (j % kStages) * kTile;
+        const uint64_t dq = sw128_desc(base + kOffQ + x * kTile, 16, 1024);
+        const uint64_t dk = sw128_desc(base + kOffK + (j % kStages) * kTile, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_bf16(tmem + x * kRows, sw128_desc(q + ks * 32, 16, 1024),
-                   sw128_desc(k + ks * 32, 16, 1024), idS, ks > 0);
+          mma_bf16(tmem + x * kRows, desc_add(dq, ks * 32), desc_add(dk, ks * 32), idS, ks > 0);
       };
       auto issue_PV = [&](int x, int j) {
-        const uint32_t p = base + kOffP + x * kPTile, v = base + kOffV + (j % kStages) * kTile;
+        const uint64_t dp = sw128_desc(base + kOffP + x * kPTile, 16, 1024);
+        const uint64_t dv = sw128_desc(base + kOffV + (j % kStages) * kTile, kTile, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + 2 * kRows + x * kD,
-                   sw128_desc(p + (kk >> 2) * (kRows * 128) + (kk & 3) * 32, 16, 1024),
-                   sw128_desc(v + kk * 2048, kTile, 1024), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16(tmem + 2 * kRows + x * kD, desc_add(dp, (kk >> 2) * (kRows * 128) + (kk & 3) * 32),
+                   desc_add(dv, kk * 2048), idPV, (j > 0 || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bars + kBarQ, 0, abort, status) && mbar_wait(bars + kBarK, 0, abort, status);
       if (ok) {
@@ -343,13 +345,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// [rows, 64] bf16 row-major, tiles of 128 rows x 64 columns, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows) {
+// [rows, 64] bf16 row-major, tiles of box_rows rows x 64 columns, 128-byte
+// swizzle.
+bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)kRows};
+  cuuint32_t box[2] = {(cuuint32_t)kD, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -359,8 +362,8 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows) {
 cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                void* O, float* lse, cudaStream_t st) {
   CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, Q, BH * S) || !make_tile_map(&mk, K, BH * S) ||
-      !make_tile_map(&mv, V, BH * S))
+  if (!make_tile_map(&mq, Q, BH * S, kRows) || !make_tile_map(&mk, K, BH * S, kRows) ||
+      !make_tile_map(&mv, V, BH * S, kRows))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
   static bool attr_set = false;

@@ -194,6 +194,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same descriptor advanced by `bytes` (a multiple of 16): only the start
+// address field changes, and it cannot carry out of its 14 bits for an
+// address inside shared memory, so a plain add is enough.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and an fp32 accumulator.
 // b_mn: B operand MN-major (else K-major); A is always K-major here.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn) {
