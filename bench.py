@@ -255,6 +255,20 @@ def workload_config(w, n):
 # ---------------------------------------------------------------------------
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank takes the same collective step."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job Mtok/s: all ranks' tokens over the max-over-ranks step time."""
+    return tokens_per_rank * world / (ms * 1e-3) / 1e6
+
+
 def timed_steps(layer, st, steps, backward=True):
     n = len(STAGES) if backward else 5
     start = torch.cuda.Event(enable_timing=True)
@@ -355,13 +369,11 @@ def main():
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, "cuda")
     lh.device_status()
 
     tokens = w.B * w.N * world
-    value = tokens / (ms * 1e-3) / 1e6
+    value = throughput(w.B * w.N, world, ms)
     peaks = load_peaks()
     work = stage_work(layer.pl, w)
     stages = {}
@@ -410,11 +422,7 @@ def main():
         e2e_once()
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, "cuda")
     nbytes = Q.numel() * Q.element_size()
 
     extras = {}
