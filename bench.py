@@ -388,13 +388,17 @@ def main():
                             "frac_tensor": tf / peaks["bf16_sus"]}
     dom = max(STAGES, key=lambda s: stages[s]["ms"])
     d = stages[dom]
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get(f"lh_{dom}@{w.name}")
     if "flops" in d:
         roof = {"kernel": f"lh_{dom}", "bound": "tensor", "achieved": d["TFLOP/s"],
                 "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": d["frac_tensor"],
-                "traffic": None, "peak_source": f"{peaks['src']} bf16 sustained"}
+                "traffic": traffic, "peak_source": f"{peaks['src']} bf16 sustained"}
     else:
         roof = {"kernel": f"lh_{dom}", "bound": "hbm", "achieved": d["GB/s"], "peak": peaks["hbm"],
-                "unit": "GB/s", "frac": d["frac_hbm"], "traffic": None,
+                "unit": "GB/s", "frac": d["frac_hbm"], "traffic": traffic,
                 "peak_source": f"{peaks['src']} HBM copy"}
 
     # end to end through the public API: host buffers, copies inside the timed region
