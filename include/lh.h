@@ -154,12 +154,18 @@ lh_status lh_gather(const lh_plan* plan, const void* Q, const void* K, const voi
 lh_status lh_attn_fwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, void* Og, float* lse, lh_stream_t stream);
 
-/* Bytes of scratch lh_attn_bwd needs for BH problems of length S. */
+/* Bytes of scratch lh_attn_bwd needs for BH problems of length S: the row
+ * term D (BH * S floats) and, for bf16, an fp32 dQ accumulator (BH * S * d
+ * floats), each rounded up to 256 bytes. */
 int64_t lh_attn_bwd_ws_bytes(int64_t BH, int64_t S, int32_t d, int32_t dtype);
 
 /* Gradients of lh_attn_fwd.  D: [BH, S] fp32 rowsum(dOg * Og), or NULL, in
  * which case it is computed into ws from Og and dOg.  Writes dQg, dKg, dVg
- * [BH, S, d].  ws: lh_attn_bwd_ws_bytes() bytes. */
+ * [BH, S, d].  ws: lh_attn_bwd_ws_bytes() bytes.
+ * bf16 runs one fused kernel by default: dQg is summed over key tiles with
+ * fp32 atomics, so its last bits may differ between runs (dKg and dVg are
+ * bit-reproducible).  lh_set_deterministic(1) selects a two-kernel schedule
+ * without atomics (about 1.5x the time), as does lh_attn_bwd_static. */
 lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, const void* Og, const float* lse,
                       const void* dOg, const float* D, void* dQg, void* dKg, void* dVg,
@@ -184,6 +190,12 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
  *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library
  *    call. */
 #define LH_ATTN_BWD_STATIC_MAX_ROWS (1 << 20)
+/* Process-wide switch for lh_attn_bwd and lh_backward: on != 0 makes every
+ * later bf16 attention backward bit-reproducible (two kernels, no atomics);
+ * 0 (the default) restores the fused kernel.  Affects work enqueued after
+ * the call only; thread-safe. */
+void lh_set_deterministic(int on);
+
 lh_status lh_attn_bwd_static(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                              const void* Kg, const void* Vg, const void* Og, const float* lse,
                              const void* dOg, void* dQg, void* dKg, void* dVg, lh_stream_t stream);

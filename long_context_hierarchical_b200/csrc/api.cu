@@ -271,6 +271,8 @@ lh_status lh_attn_fwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
   return ok();
 }
 
+void lh_set_deterministic(int on) { set_deterministic(on); }
+
 int64_t lh_attn_bwd_ws_bytes(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
   if (check_attn(BH, S, d, dtype) != LH_OK) return -1;
   return attn_bwd_ws_bytes(BH, S, dtype);

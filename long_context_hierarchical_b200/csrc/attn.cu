@@ -1,4 +1,6 @@
 // Stage-3 attention dispatch: the storage dtype picks the kernel family.
+#include <atomic>
+
 #include "host.h"
 
 namespace lh {
@@ -14,11 +16,21 @@ cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void*
                                void* O, float* lse, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                const float* lse, const void* dO, const float* D, void* dQ,
-                               void* dK, void* dV, cudaStream_t st);
+                               void* dK, void* dV, float* dq_acc, cudaStream_t st);
 
+namespace {
+std::atomic<int> g_deterministic{0};
+int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+}  // namespace
+
+void set_deterministic(int on) { g_deterministic.store(on != 0); }
+int deterministic() { return g_deterministic.load(); }
+
+// [D when the caller passes none | bf16: fp32 dQ accumulator of the fused
+// schedule, BH * S * 64 floats]
 int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype) {
-  (void)dtype;
-  return ((BH * S * 4) + 255) & ~int64_t(255);  // D when the caller passes none
+  const int64_t d_bytes = align256(BH * S * 4);
+  return dtype == LH_BF16 ? d_bytes + align256(BH * S * kD * 4) : d_bytes;
 }
 
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
@@ -42,7 +54,12 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, co
   if (dtype == LH_F32)
     return launch_attn_bwd_f32(BH, S, (const float*)Qg, (const float*)Kg, (const float*)Vg, lse,
                                (const float*)dOg, D, (float*)dQg, (float*)dKg, (float*)dVg, st);
-  return launch_attn_bwd_tc(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, st);
+  // Without a workspace (the allocation-free entry point) or in deterministic
+  // mode the two-kernel schedule runs; otherwise the fused one.
+  float* dq_acc = (ws != nullptr && !deterministic())
+                      ? reinterpret_cast<float*>(static_cast<char*>(ws) + align256(BH * S * 4))
+                      : nullptr;
+  return launch_attn_bwd_tc(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, dq_acc, st);
 }
 
 }  // namespace lh

@@ -5,14 +5,22 @@
 // With P = exp(s - lse) from the forward's LSE, dP = dO V^T and
 // dS = P (dP - D), D = rowsum(dO O):
 //   dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d).
-// Two kernels, deterministic, no atomics:
-//  - dk/dv: one CTA per 128-key tile streams query chunks of C rows from its
-//    diagonal on.  S^T = K Q^T and dP^T = V dO^T land in TMEM (lane = key);
-//    the element-wise warps turn them into P^T and dS^T (bf16, swizzled
-//    K-major smem); dV += P^T dO and dK += dS^T Q accumulate in TMEM.
-//  - dq: one CTA per 128-query tile streams key chunks of C rows up to its
-//    diagonal.  S = Q K^T and dP = dO V^T in TMEM (lane = query), dS to smem,
-//    dQ += dS K in TMEM.
+// Two schedules:
+//  - fused (default): one kernel.  A CTA per 128-key tile streams query
+//    chunks of C rows from its diagonal on.  S^T = K Q^T and dP^T = V dO^T
+//    land in TMEM (lane = key); the element-wise warps turn them into P^T
+//    and dS^T (bf16, swizzled K-major smem); dV += P^T dO and dK += dS^T Q
+//    accumulate in TMEM, and the chunk's dQ share dS K (the dS^T tile read
+//    MN-major as the A operand) lands in TMEM, from where the element-wise
+//    warps add it into an fp32 dQ accumulator in global memory (fp32
+//    atomics, so the summation order, and the last bits of dQ, vary from
+//    run to run).  A small kernel scales and rounds the accumulator to dQ.
+//    P and dS are formed once per (key, query) pair.
+//  - deterministic: two kernels, no atomics.  The dk/dv kernel above without
+//    the dQ share, then a dq kernel: one CTA per 128-query tile streams key
+//    chunks of C rows up to its diagonal; S = Q K^T and dP = dO V^T in TMEM
+//    (lane = query), dS to smem, dQ += dS K in TMEM.  P and dS are formed
+//    twice.
 // Warp roles: C/32 element-wise groups of four warps split each step's C
 // columns (no row reductions are needed here), then one load warp (TMA for
 // tiles, plain loads for LSE/D) and one warp that owns TMEM and issues the
@@ -27,12 +35,15 @@
 // Operand layouts are those of the forward kernel: K-major A/B tiles with the
 // 128-byte swizzle, tiles read as the MN-major B operand (dO, Q, K) with
 // 8-row groups 1024 bytes apart.  Every wait is bounded (see tc.cuh).
+#include <algorithm>
+
 #include "host.h"
 #include "tc.cuh"
 
 namespace lh {
 
 bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows);
+bool make_acc_map(CUtensorMap* map, const float* ptr, int64_t rows);
 
 namespace {
 
@@ -113,34 +124,97 @@ __device__ __forceinline__ void gemm_acc(uint32_t d, uint32_t a, uint32_t b, boo
              (acc || kk > 0) ? 1u : 0u);
 }
 
+// D[tmem] = dS(128 queries x 128 keys) * K(128 keys x 64): A is the dS^T tile
+// (K-major for the dK product) read MN-major, its two 64-query column blocks
+// kKBlock apart; B is the resident K tile read MN-major.
+__device__ __forceinline__ void gemm_dq(uint32_t d, uint32_t dst_tile, uint32_t k_tile) {
+  constexpr uint32_t idesc = idesc_bf16(kRows, kD, true, true);
+  const uint64_t da = sw128_desc(dst_tile, kKBlock, 1024), db = sw128_desc(k_tile, kTileR, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kRows / 16; ++kk)
+    mma_bf16(d, desc_add(da, kk * 2048), desc_add(db, kk * 2048), idesc, kk > 0 ? 1u : 0u);
+}
+
+// D[tmem] (+)= A(128 x C, bf16 in TMEM at a_tmem) * B(C x 64 tile read MN-major)
+template <int C>
+__device__ __forceinline__ void gemm_acc_ts(uint32_t d, uint32_t a_tmem, uint32_t b, bool acc) {
+  constexpr uint32_t idesc = idesc_bf16(kRows, kD, true);
+  const uint64_t db = sw128_desc(b, Cfg<C>::kTileC, 1024);
+#pragma unroll
+  for (int kk = 0; kk < C / 16; ++kk)
+    mma_bf16_ts(d, a_tmem + 8 * kk, desc_add(db, kk * 2048), idesc, (acc || kk > 0) ? 1u : 0u);
+}
+
 // ===========================================================================
-// dK, dV
+// dK, dV (and, fused, the dQ shares)
 // ===========================================================================
+// TMEM columns: S^T [0,C), dP^T [C,2C), dV [2C,2C+64), dK [2C+64,2C+128),
+// the chunk's dQ share [2C+128, 2C+192) (fused), P^T as bf16 pairs
+// [2C+192, 2C+192+C/2) (the A operand of dV += P^T dO).
+// Shared memory: K, V tiles; kStages x (Q chunk, dO chunk); dS^T (K-major,
+// also read MN-major by the dQ product); the dQ staging area: four boxes of
+// 128 rows x 16 fp32 (64-byte swizzle), one per element-wise group, each
+// reduced into the fp32 accumulator by one TMA reduce-add.
 template <int C>
 struct KV {
   using F = Cfg<C>;
   static constexpr uint32_t kOffK = 0, kOffV = kTileR;
-  static constexpr uint32_t kOffQ = 2 * kTileR;                       // kStages tiles
-  static constexpr uint32_t kOffG = kOffQ + F::kStages * F::kTileC;   // dO, kStages tiles
-  static constexpr uint32_t kOffPT = kOffG + F::kStages * F::kTileC;  // P^T  (128 x C)
-  static constexpr uint32_t kOffDST = kOffPT + F::kWide;              // dS^T (128 x C)
-  static constexpr uint32_t kOffVec = kOffDST + F::kWide;             // kStages x (C lse2 + C D)
+  static constexpr uint32_t kOffQ = 2 * kTileR;                        // kStages tiles
+  static constexpr uint32_t kOffG = kOffQ + F::kStages * F::kTileC;    // dO, kStages tiles
+  static constexpr uint32_t kOffDST = kOffG + F::kStages * F::kTileC;  // dS^T (128 x C)
+  static constexpr uint32_t kOffStage = kOffDST + F::kWide;            // 4 x 8 KB dQ boxes
+  static constexpr uint32_t kStageBox = kRows * 16 * 4;
+  static constexpr uint32_t kOffVec = kOffStage + 4 * kStageBox;       // kStages x (C lse2 + C D)
   static constexpr uint32_t kOffBar = kOffVec + F::kStages * 2 * C * 4;
   static constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * F::kStages,
                             kBarSP = kBarEmpty + 8 * F::kStages, kBarPDS = kBarSP + 8,
                             kBarAcc = kBarPDS + 8, kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8,
-                            kBarPF = kBarTF + 8, kSlotTmem = kBarPF + 8, kSlotAbort = kSlotTmem + 4;
+                            kBarPF = kBarTF + 8, kBarStaged = kBarPF + 8,
+                            kSlotTmem = kBarStaged + 8 * 4, kSlotAbort = kSlotTmem + 4;
   static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-  static constexpr uint32_t kTmemCols = pow2_cols(2 * C + 2 * kD);
+  static constexpr uint32_t kColDQ = 2 * C + 2 * kD;
+  static constexpr uint32_t kColPT = 2 * C + 3 * kD;
+  static constexpr uint32_t kTmemCols = pow2_cols(kColPT + C / 2);
+  static_assert(kColPT + C / 2 <= 512, "TMEM columns");
+  static_assert(kOffBar + 256 <= 227 * 1024, "shared memory");
 };
 
-template <int C>
+// One element-wise group's part of a chunk's dQ share: this thread's 16
+// columns of its query row (TMEM lane) into the group's staging box, then the
+// group's first lane reduces the box into rows [q_first, q_first + 128) of
+// the fp32 accumulator.  The box is free: the previous reduce from it
+// finished reading before its issuer's last arrival on the P/dS barrier,
+// which precedes the completion this thread waited for.  Rows past S add
+// the zeros of masked dS (or fall past the tensor and are dropped).
+__device__ __forceinline__ bool stage_dq16(uint32_t taddr, uint32_t box, int rq, uint32_t staged,
+                                           uint32_t parity, bool issuer, const CUtensorMap* map,
+                                           int x, int y, volatile int* abort,
+                                           unsigned int* status) {
+  float v[16];
+  tmem_ld16(taddr, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t w[4] = {__float_as_uint(v[4 * c]), __float_as_uint(v[4 * c + 1]),
+                           __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3])};
+    st_shared_v4(box + rq * 64 + ((c ^ ((rq >> 1) & 3)) << 4), w);
+  }
+  fence_proxy_async();
+  mbar_arrive(staged);
+  if (!issuer) return true;
+  if (!mbar_wait(staged, parity, abort, status)) return false;
+  tma_reduce_add_2d(map, x, y, box);
+  return true;
+}
+
+template <int C, bool kFused>
 __global__ void __launch_bounds__(Cfg<C>::kThreads, Cfg<C>::kCtas)
 attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
-                        const float* __restrict__ lse, const float* __restrict__ Dv,
-                        bf16* __restrict__ dK, bf16* __restrict__ dV, int S, float sl2, float scale,
-                        unsigned int* __restrict__ status) {
+                        const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
+                        const float* __restrict__ Dv, bf16* __restrict__ dK, bf16* __restrict__ dV,
+                        int S, float sl2, float scale, unsigned int* __restrict__ status) {
+  static_assert(C == kRows, "a dQ share has one TMEM lane per query of the chunk");
   using F = Cfg<C>;
   using L = KV<C>;
   extern __shared__ uint8_t smem_raw[];
@@ -169,7 +243,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     mbar_init(bars + L::kBarAcc, 1);
     mbar_init(bars + L::kBarDrain, 1);
     mbar_init(bars + L::kBarTF, F::kEw);  // S^T/dP^T copied out of TMEM
-    mbar_init(bars + L::kBarPF, 1);       // P^T/dS^T tile consumed by the MMAs
+    mbar_init(bars + L::kBarPF, 1);       // P^T/dS^T (and the dQ share) consumed / complete
+    for (int g = 0; g < 4; ++g) mbar_init(bars + L::kBarStaged + 8 * g, 128);
     *abort = 0;
     fence_mbar_init();
   }
@@ -240,8 +315,9 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         if (!(ok = mbar_wait(bars + L::kBarPDS, t & 1, abort, status))) break;
         tc_fence_after();
-        gemm_acc<C>(tmem + 2 * C, base + L::kOffPT, base + L::kOffG + s * F::kTileC, t > 0);       // dV += P^T dO
+        gemm_acc_ts<C>(tmem + 2 * C, tmem + L::kColPT, base + L::kOffG + s * F::kTileC, t > 0);  // dV += P^T dO
         gemm_acc<C>(tmem + 2 * C + kD, base + L::kOffDST, base + L::kOffQ + s * F::kTileC, t > 0); // dK += dS^T Q
+        if constexpr (kFused) gemm_dq(tmem + L::kColDQ, base + L::kOffDST, base + L::kOffK);  // dS K
         mma_commit(bars + L::kBarPF);
         mma_commit(bars + L::kBarEmpty + 8 * s);
       }
@@ -250,12 +326,15 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       wait_drain(bars + L::kBarDrain, 0);
     }
   } else {
-    // ---------------- element-wise: P^T, dS^T ----------------
+    // ---------------- element-wise: P^T, dS^T (and the dQ shares) ----------------
     const int grp = warp >> 2, wr = warp & 3;
-    const int r = wr * 32 + lane;  // key row of the tile = TMEM lane
+    const int r = wr * 32 + lane;  // TMEM lane: key row of the tile, query row of a dQ share
     const int key = k0 + r;
     const int col0 = grp * 32;     // this group's 32 query columns of the step
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
+    const bool issuer = kFused && wr == 0 && lane == 0;
+    const uint32_t staged = bars + L::kBarStaged + 8 * grp;
+    const uint32_t box = base + L::kOffStage + grp * L::kStageBox;
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
@@ -295,19 +374,35 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         wd[e >> 1] = pack_bf16x2(p[0] * (dp[e] - dv.x), p[1] * (dp[e + 1] - dv.y));
         wd[(e >> 1) + 1] = pack_bf16x2(p[2] * (dp[e + 2] - dv.z), p[3] * (dp[e + 3] - dv.w));
       }
-      // the previous step's P^T / dS^T must be consumed before they are overwritten
+      // the previous step's P^T / dS^T (and dQ share) must be consumed before
+      // they are overwritten
       if (t > 0) ok = mbar_wait(bars + L::kBarPF, (t - 1) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      store_row32(base + L::kOffPT, r, grp, wp);
+      tc_fence_after();
+      tmem_st16(lane_base + L::kColPT + 16 * grp, wp);
+      if constexpr (kFused) {
+        if (t > 0) {
+          ok = stage_dq16(lane_base + L::kColDQ + 16 * grp, box, r, staged, (t - 1) & 1, issuer, &tmDQ,
+                          16 * grp, row0 + q0 - C, abort, status);
+        }
+      }
       store_row32(base + L::kOffDST, r, grp, wd);
       fence_proxy_async();
+      if (issuer) bulk_wait_read();  // the staging box is free before the next P/dS arrival
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + L::kBarPDS);
+      if (!__all_sync(0xffffffffu, ok)) break;
     }
     if (ok) ok = mbar_wait(bars + L::kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
-      // TMEM [2C, 2C+64) = dV, [2C+64, 2C+128) = dK: 128 columns over the groups
       tc_fence_after();
+      if constexpr (kFused) {
+        if (nq > 0)
+          stage_dq16(lane_base + L::kColDQ + 16 * grp, box, r, staged, (nq - 1) & 1, issuer, &tmDQ,
+                     16 * grp, row0 + k0 + (nq - 1) * C, abort, status);
+      }
+      // TMEM [2C, 2C+64) = dV, [2C+64, 2C+128) = dK: 128 columns over the groups
 #pragma unroll
       for (int piece = 0; piece < 4 / F::kGroups; ++piece) {
         const int c = (grp * (4 / F::kGroups) + piece) * 32;  // 0..127
@@ -321,6 +416,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
       }
     }
+    if (issuer) bulk_wait_all();  // the reduces are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -512,13 +608,25 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   }
 }
 
+// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
+__global__ void __launch_bounds__(256) dq_round_kernel(const float4* __restrict__ acc,
+                                                       uint4* __restrict__ dQ, int64_t n8,
+                                                       float scale) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldcs(acc + 2 * i), b = __ldcs(acc + 2 * i + 1);
+    __stcs(dQ + i, make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                              pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale)));
+  }
+}
+
 constexpr int kStep = 128;  // streamed rows per step (64 measured slower: N=64 MMAs run at ~65% rate)
 
 }  // namespace
 
 cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                const float* lse, const void* dO, const float* D, void* dQ,
-                               void* dK, void* dV, cudaStream_t st) {
+                               void* dK, void* dV, float* dq_acc, cudaStream_t st) {
   constexpr int C = kStep;
   using F = Cfg<C>;
   // Tiles that stay resident in a CTA have 128 rows; streamed chunks have C.
@@ -532,8 +640,11 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   unsigned int* status = device_status_ptr();
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<C>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<C, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, KV<C>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<C, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, KV<C>::kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              QQ<C>::kSmemBytes);
@@ -543,9 +654,26 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float sl2 = 0.125f * kLog2e;
   const dim3 grid(ntiles, (unsigned)BH);
-  attn_bwd_dkdv_tc_kernel<C><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
-      qC, kR, vR, gC, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2, 0.125f,
-      status);
+  if (dq_acc != nullptr) {
+    const int64_t n = BH * S * kD;
+    CUtensorMap accM;
+    if (!make_acc_map(&accM, dq_acc, rows)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)n * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    attn_bwd_dkdv_tc_kernel<C, true><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
+        qC, kR, vR, gC, accM, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2,
+        0.125f, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int64_t n8 = n / 8;
+    const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
+    dq_round_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
+                                            static_cast<uint4*>(dQ), n8, 0.125f);
+    return cudaGetLastError();
+  }
+  attn_bwd_dkdv_tc_kernel<C, false><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
+      qC, kR, vR, gC, qC /* no dQ shares */, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV),
+      (int)S, sl2, 0.125f, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dq_tc_kernel<C><<<grid, F::kThreads, QQ<C>::kSmemBytes, st>>>(

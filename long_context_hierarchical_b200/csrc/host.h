@@ -43,6 +43,8 @@ cudaError_t launch_gather_bwd(const lh_plan& plan, const void* dQg, const void* 
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
                             const void* Vg, void* Og, float* lse, cudaStream_t st);
 int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype);
+void set_deterministic(int on);
+int deterministic();
 cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
                             const void* Vg, const void* Og, const float* lse, const void* dOg,
                             const float* D, void* dQg, void* dKg, void* dVg, void* ws,

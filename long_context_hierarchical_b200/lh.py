@@ -26,7 +26,7 @@ EXPORTS = (
     "lh_plan_init", "lh_pyramid", "lh_score", "lh_pyramid_score", "lh_topk", "lh_gather",
     "lh_attn_fwd", "lh_attn_bwd_ws_bytes", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd",
     "lh_gather_bwd", "lh_forward", "lh_backward", "lh_device_status", "lh_status_string",
-    "lh_last_error", "lh_plan_bytes", "lh_attn_bwd_static",
+    "lh_last_error", "lh_plan_bytes", "lh_attn_bwd_static", "lh_set_deterministic",
 )
 
 
@@ -95,6 +95,8 @@ def _load():
     lib.lh_last_error.restype = ctypes.c_char_p
     lib.lh_plan_bytes.argtypes = []
     lib.lh_plan_bytes.restype = I64
+    lib.lh_set_deterministic.argtypes = [ctypes.c_int]
+    lib.lh_set_deterministic.restype = None
     if lib.lh_plan_bytes() != ctypes.sizeof(LhPlan):
         raise ImportError("lh_plan layout of liblh.so does not match this binding")
     return lib
@@ -353,6 +355,12 @@ def backward(pl: Plan, dO, ctx: Context, dQ=None, dK=None, dV=None, ws: Workspac
     _check(LIB.lh_backward(pl.byref(), _ptr(dO), _ptr(ctx.buf), _ptr(dQ), _ptr(dK), _ptr(dV),
                            _ptr(ws.buf), _stream(stream)), "lh_backward")
     return dQ, dK, dV
+
+
+def set_deterministic(on: bool):
+    """Process-wide: bit-reproducible bf16 attention backward (two kernels, no
+    atomics) for lh_attn_bwd / lh_backward calls enqueued afterwards."""
+    LIB.lh_set_deterministic(1 if on else 0)
 
 
 def device_status(reset: bool = True):

@@ -166,17 +166,50 @@ def test_scatter_backward(case):
     assert_close(np64(D), _grad_stack(c, "D"), dt, "D")
 
 
-def test_attention_backward(case):
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_attention_backward(case, deterministic):
     c = case
     lh, dt = c["lh"], c["dt"]
     Qg, Kg, Vg, Og = (_t(stack(c["ctxs"], k), dt) for k in ("Qg", "Kg", "Vg", "Og"))
     lse = _t(stack(c["ctxs"], "lse"), torch.float32)
     dOg = _t(_grad_stack(c, "dOg"), dt)
     D = _t(_grad_stack(c, "D"), torch.float32)
-    for Din in (D, None):
-        dQg, dKg, dVg = lh.attn_bwd(Qg, Kg, Vg, Og, lse, dOg, Din)
-        for got, key in ((dQg, "dQg"), (dKg, "dKg"), (dVg, "dVg")):
-            assert_grad_close(np64(got), _grad_stack(c, key), c["terms"][key], dt, key)
+    lh.set_deterministic(deterministic)
+    try:
+        for Din in (D, None):
+            dQg, dKg, dVg = lh.attn_bwd(Qg, Kg, Vg, Og, lse, dOg, Din)
+            for got, key in ((dQg, "dQg"), (dKg, "dKg"), (dVg, "dVg")):
+                assert_grad_close(np64(got), _grad_stack(c, key), c["terms"][key], dt, key)
+    finally:
+        lh.set_deterministic(False)
+    lh.device_status()
+
+
+def test_attention_backward_schedules_agree(case):
+    """The fused schedule (dQ shares added with fp32 atomics) and the
+    deterministic two-kernel one: dK, dV from the same kernel code are
+    bit-identical, dQ differs only by the order of its fp32 sum; the
+    deterministic schedule repeats bit for bit."""
+    c = case
+    lh, dt = c["lh"], c["dt"]
+    Qg, Kg, Vg, Og = (_t(stack(c["ctxs"], k), dt) for k in ("Qg", "Kg", "Vg", "Og"))
+    lse = _t(stack(c["ctxs"], "lse"), torch.float32)
+    dOg = _t(_grad_stack(c, "dOg"), dt)
+    fused = lh.attn_bwd(Qg, Kg, Vg, Og, lse, dOg, None)
+    lh.set_deterministic(True)
+    try:
+        det = [lh.attn_bwd(Qg, Kg, Vg, Og, lse, dOg, None) for _ in range(2)]
+    finally:
+        lh.set_deterministic(False)
+    for a, b in zip(det[0], det[1]):
+        assert torch.equal(a, b)
+    assert torch.equal(fused[1], det[0][1]) and torch.equal(fused[2], det[0][2])
+    a, b = np64(fused[0]), np64(det[0][0])
+    # both are fp32 sums of the same shares rounded once: at most one rounding
+    # step of the output type apart, plus fp32 reordering under cancellation
+    step = 2.0 ** -7 if dt == torch.bfloat16 else 2.0 ** -22
+    tq = c["terms"]["dQg"]
+    assert np.all(np.abs(a - b) <= step * np.abs(b) + 2.0 ** -14 * tq + 1e-30), "dQg fused vs deterministic"
 
 
 def test_gather_backward(case):
@@ -200,11 +233,21 @@ def test_whole_layer(case):
     assert_grad_close(np64(O), c["O"], c["terms"]["O"], dt, "O")
     for got, i, key in ((dQ, 0, "dQ"), (dK, 1, "dK"), (dV, 2, "dV")):
         assert_grad_close(np64(got), c["grads"][i], c["terms"][key], dt, key)
-    # run to run: bit-identical
+    # run to run: the forward, dK and dV bit-identical (the default fused
+    # backward sums dQ with fp32 atomics); everything in deterministic mode
     O2, ctx2 = lh.forward(pl, c["Q"], c["K"], c["V"])
     g2 = lh.backward(pl, c["dO"], ctx2)
     assert torch.equal(O, O2)
-    for a, b in zip((dQ, dK, dV), g2):
+    assert torch.equal(dK, g2[1]) and torch.equal(dV, g2[2])
+    lh.set_deterministic(True)
+    try:
+        g3 = lh.backward(pl, c["dO"], ctx2)
+        g4 = lh.backward(pl, c["dO"], ctx2)
+    finally:
+        lh.set_deterministic(False)
+    for got, i, key in ((g3[0], 0, "dQ"), (g3[1], 1, "dK"), (g3[2], 2, "dV")):
+        assert_grad_close(np64(got), c["grads"][i], c["terms"][key], dt, key)
+    for a, b in zip(g3, g4):
         assert torch.equal(a, b)
     lh.device_status()
 
