@@ -169,8 +169,8 @@ struct KV {
   static constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * F::kStages,
                             kBarSP = kBarEmpty + 8 * F::kStages, kBarPDS = kBarSP + 8,
                             kBarAcc = kBarPDS + 8, kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8,
-                            kBarPF = kBarTF + 8, kBarStaged = kBarPF + 8,
-                            kSlotTmem = kBarStaged + 8 * 4, kSlotAbort = kSlotTmem + 4;
+                            kBarPF = kBarTF + 8, kBarQD = kBarPF + 8, kBarBF = kBarQD + 8,
+                            kSlotTmem = kBarBF + 8, kSlotAbort = kSlotTmem + 4;
   static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
   static constexpr uint32_t kColDQ = 2 * C + 2 * kD;
   static constexpr uint32_t kColPT = 2 * C + 3 * kD;
@@ -179,17 +179,10 @@ struct KV {
   static_assert(kOffBar + 256 <= 227 * 1024, "shared memory");
 };
 
-// One element-wise group's part of a chunk's dQ share: this thread's 16
-// columns of its query row (TMEM lane) into the group's staging box, then the
-// group's first lane reduces the box into rows [q_first, q_first + 128) of
-// the fp32 accumulator.  The box is free: the previous reduce from it
-// finished reading before its issuer's last arrival on the P/dS barrier,
-// which precedes the completion this thread waited for.  Rows past S add
-// the zeros of masked dS (or fall past the tensor and are dropped).
-__device__ __forceinline__ bool stage_dq16(uint32_t taddr, uint32_t box, int rq, uint32_t staged,
-                                           uint32_t parity, bool issuer, const CUtensorMap* map,
-                                           int x, int y, volatile int* abort,
-                                           unsigned int* status) {
+// This thread's 16 columns of its query row (TMEM lane) of a chunk's dQ
+// share into its group's staging box (64-byte swizzle: the 16-byte chunk c
+// of row r sits at chunk c ^ ((r >> 1) & 3)).
+__device__ __forceinline__ void stage_dq16(uint32_t taddr, uint32_t box, int rq) {
   float v[16];
   tmem_ld16(taddr, v);
   tmem_wait_ld();
@@ -199,16 +192,12 @@ __device__ __forceinline__ bool stage_dq16(uint32_t taddr, uint32_t box, int rq,
                            __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3])};
     st_shared_v4(box + rq * 64 + ((c ^ ((rq >> 1) & 3)) << 4), w);
   }
-  fence_proxy_async();
-  mbar_arrive(staged);
-  if (!issuer) return true;
-  if (!mbar_wait(staged, parity, abort, status)) return false;
-  tma_reduce_add_2d(map, x, y, box);
-  return true;
 }
 
+// 18 warps: five of them share one SM sub-partition's 16K registers, so 96
+// registers per thread is the most a launch can have.
 template <int C, bool kFused>
-__global__ void __launch_bounds__(Cfg<C>::kThreads, Cfg<C>::kCtas)
+__global__ void __launch_bounds__(Cfg<C>::kThreads, 1)
 attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                         const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
@@ -244,7 +233,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     mbar_init(bars + L::kBarDrain, 1);
     mbar_init(bars + L::kBarTF, F::kEw);  // S^T/dP^T copied out of TMEM
     mbar_init(bars + L::kBarPF, 1);       // P^T/dS^T (and the dQ share) consumed / complete
-    for (int g = 0; g < 4; ++g) mbar_init(bars + L::kBarStaged + 8 * g, 128);
+    mbar_init(bars + L::kBarQD, F::kEw);  // a dQ share read out of TMEM and staged
+    mbar_init(bars + L::kBarBF, 1);       // the staging boxes read by the last reduce
     *abort = 0;
     fence_mbar_init();
   }
@@ -301,6 +291,14 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG, idS);  // dP^T = V dO^T
         mma_commit(bars + L::kBarSP);
       }
+      // dQ share j: issued as step j's last MMA, staged by the element-wise
+      // warps after step j+1's P/dS hand-off (QD), reduced from here into
+      // rows [k0 + C j, +C) of the accumulator; its boxes are released (BF)
+      // one step later.
+      auto reduce_share = [&](int j) {
+        for (int g = 0; g < 4; ++g)
+          tma_reduce_add_2d(&tmDQ, 16 * g, row0 + k0 + j * C, base + L::kOffStage + g * L::kStageBox);
+      };
       for (int t = 0; ok && t < nq; ++t) {
         const int s = t % F::kStages;
         // S^T/dP^T of step t copied out: start step t+1's while step t computes
@@ -313,15 +311,36 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
           gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG + s1 * F::kTileC, idS);
           mma_commit(bars + L::kBarSP);
         }
+        if constexpr (kFused) {
+          if (t >= 2) {  // share t-2's reduce has read the boxes
+            bulk_wait_read();
+            mbar_arrive(bars + L::kBarBF);
+          }
+        }
         if (!(ok = mbar_wait(bars + L::kBarPDS, t & 1, abort, status))) break;
         tc_fence_after();
         gemm_acc_ts<C>(tmem + 2 * C, tmem + L::kColPT, base + L::kOffG + s * F::kTileC, t > 0);  // dV += P^T dO
         gemm_acc<C>(tmem + 2 * C + kD, base + L::kOffDST, base + L::kOffQ + s * F::kTileC, t > 0); // dK += dS^T Q
-        if constexpr (kFused) gemm_dq(tmem + L::kColDQ, base + L::kOffDST, base + L::kOffK);  // dS K
+        if constexpr (kFused) {
+          if (t >= 1) {  // share t-1 out of TMEM and staged
+            if (!(ok = mbar_wait(bars + L::kBarQD, (t - 1) & 1, abort, status))) break;
+            tc_fence_after();
+            reduce_share(t - 1);
+          }
+          gemm_dq(tmem + L::kColDQ, base + L::kOffDST, base + L::kOffK);  // share t = dS K
+        }
         mma_commit(bars + L::kBarPF);
         mma_commit(bars + L::kBarEmpty + 8 * s);
       }
       if (ok) mma_commit(bars + L::kBarAcc);
+      if constexpr (kFused) {
+        if (ok && nq >= 2) {
+          bulk_wait_read();
+          mbar_arrive(bars + L::kBarBF);
+        }
+        if (ok && mbar_wait(bars + L::kBarQD, (nq - 1) & 1, abort, status)) reduce_share(nq - 1);
+        bulk_wait_all();  // the reduces are complete before the CTA exits
+      }
       mma_commit(bars + L::kBarDrain);
       wait_drain(bars + L::kBarDrain, 0);
     }
@@ -332,9 +351,16 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     const int key = k0 + r;
     const int col0 = grp * 32;     // this group's 32 query columns of the step
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
-    const bool issuer = kFused && wr == 0 && lane == 0;
-    const uint32_t staged = bars + L::kBarStaged + 8 * grp;
     const uint32_t box = base + L::kOffStage + grp * L::kStageBox;
+    // share j: wait until share j-1's reduce has read the boxes, stage, arrive
+    auto stage_share = [&](int j) -> bool {
+      if (j >= 1 && !mbar_wait(bars + L::kBarBF, (j - 1) & 1, abort, status)) return false;
+      stage_dq16(lane_base + L::kColDQ + 16 * grp, box, r);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bars + L::kBarQD);
+      return true;
+    };
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
@@ -380,27 +406,22 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
       tmem_st16(lane_base + L::kColPT + 16 * grp, wp);
-      if constexpr (kFused) {
-        if (t > 0) {
-          ok = stage_dq16(lane_base + L::kColDQ + 16 * grp, box, r, staged, (t - 1) & 1, issuer, &tmDQ,
-                          16 * grp, row0 + q0 - C, abort, status);
-        }
-      }
       store_row32(base + L::kOffDST, r, grp, wd);
       fence_proxy_async();
-      if (issuer) bulk_wait_read();  // the staging box is free before the next P/dS arrival
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + L::kBarPDS);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if constexpr (kFused) {
+        // share t-1 (complete: PF above) leaves TMEM while dV/dK of step t run
+        if (t >= 1) ok = stage_share(t - 1);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      }
     }
     if (ok) ok = mbar_wait(bars + L::kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       if constexpr (kFused) {
-        if (nq > 0)
-          stage_dq16(lane_base + L::kColDQ + 16 * grp, box, r, staged, (nq - 1) & 1, issuer, &tmDQ,
-                     16 * grp, row0 + k0 + (nq - 1) * C, abort, status);
+        if (nq > 0) stage_share(nq - 1);
       }
       // TMEM [2C, 2C+64) = dV, [2C+64, 2C+128) = dK: 128 columns over the groups
 #pragma unroll
@@ -416,7 +437,6 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
       }
     }
-    if (issuer) bulk_wait_all();  // the reduces are complete before the CTA exits
   }
 
   tc_fence_before();

@@ -11,13 +11,15 @@
 //              exchange of the two halves' maxima through shared memory;
 //   warp 16    TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
 //   warp 17    TMEM allocation and the single MMA-issuing thread.
-// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384),
-// fp32.  Per key tile j the MMA thread issues S_X = Q_X K_j^T (M=128, N=128,
-// 4 x K=16) and, once softmax X has written P_X (bf16, swizzled K-major smem),
-// O_X += P_X V_j (M=128, N=64, 8 x K=16, V read MN-major).  The two tiles
-// ping-pong so the tensor core works on one tile while the other's softmax
-// runs.  O is rescaled in TMEM only when a row maximum grows by more than
-// 2^8 (the reference maximum otherwise stays, so P <= 256).
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384)
+// fp32; P_A [384,448), P_B [448,512) as bf16 pairs.  Per key tile j the MMA
+// thread issues S_X = Q_X K_j^T (M=128, N=128, 4 x K=16) and, once softmax X
+// has written P_X into TMEM, O_X += P_X V_j (A from TMEM, V read MN-major).
+// Softmax X releases S_X as soon as it has read it (before its
+// exponentials), so S_X for tile j+1 is computed while it works on tile j;
+// it waits for the previous P V product only before overwriting P_X (or
+// rescaling O_X).  O is rescaled in TMEM only when a row maximum grows by
+// more than 2^8 (the reference maximum otherwise stays, so P <= 256).
 //
 // Every wait is bounded: on timeout the CTA records LH_ERR_TIMEOUT in the
 // device status word, stops issuing work, drains its own TMA copies and frees
@@ -36,27 +38,28 @@ using namespace tc;
 constexpr int kRows = 128;                    // query rows per tile, keys per tile
 constexpr int kStages = 3;
 constexpr uint32_t kTile = kRows * kD * 2;    // 16 KB: 128 rows x 128 B
-constexpr uint32_t kPTile = kRows * kRows * 2;  // 32 KB
 constexpr int kLoadWarp = 16, kMmaWarp = 17;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;              // log2 units
+constexpr uint32_t kColO = 2 * kRows, kColP = 2 * kRows + 2 * kD;  // TMEM columns
 
 // Shared-memory map (offsets from a 1024-byte aligned base).
 constexpr uint32_t kOffQ = 0;                          // 2 tiles
 constexpr uint32_t kOffK = kOffQ + 2 * kTile;          // kStages tiles
 constexpr uint32_t kOffV = kOffK + kStages * kTile;    // kStages tiles
-constexpr uint32_t kOffP = kOffV + kStages * kTile;    // 2 P tiles
-constexpr uint32_t kOffBar = kOffP + 2 * kPTile;
+constexpr uint32_t kOffBar = kOffV + kStages * kTile;
+// per tile x (8 bytes apart): S ready, S freed, P written, P V done
 constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
-                   kBarS = kBarE + 8 * kStages, kBarP = kBarS + 16, kBarO = kBarP + 16,
-                   kBarDrain = kBarO + 16, kBarRed = kBarDrain + 8, kBarL = kBarRed + 32,
-                   kSlotTmem = kBarL + 16, kSlotAbort = kSlotTmem + 4;
+                   kBarS = kBarE + 8 * kStages, kBarSF = kBarS + 16, kBarP = kBarSF + 16,
+                   kBarPV = kBarP + 16, kBarDrain = kBarPV + 16, kBarRed = kBarDrain + 8,
+                   kBarL = kBarRed + 32, kSlotTmem = kBarL + 16, kSlotAbort = kSlotTmem + 4;
 // Row-max exchange between the two column halves: [parity][tile][half][row];
 // then the row-sum exchange: [tile][half][row].
 constexpr uint32_t kOffRed = kOffBar + 256;
 constexpr uint32_t kOffL = kOffRed + 2 * 2 * 2 * kRows * 4;
 constexpr uint32_t kSmemBytes = kOffL + 2 * 2 * kRows * 4 + 1024;  // + alignment slack
+static_assert(kSlotAbort + 4 <= 256, "barrier area");
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   // Bounded wait that ignores the abort flag (used to drain own copies).
@@ -66,6 +69,8 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// 18 warps: five of them share one SM sub-partition's 16K registers, so 96
+// registers per thread is the most a launch can have.
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ O,
@@ -94,8 +99,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bars + kBarS + 8 * x, 1);
+      mbar_init(bars + kBarSF + 8 * x, 256);
       mbar_init(bars + kBarP + 8 * x, 256);
-      mbar_init(bars + kBarO + 8 * x, 1);
+      mbar_init(bars + kBarPV + 8 * x, 1);
       mbar_init(bars + kBarRed + 16 * x, 256);
       mbar_init(bars + kBarRed + 16 * x + 8, 256);
       mbar_init(bars + kBarL + 8 * x, 256);
@@ -148,53 +154,41 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_bf16(tmem + x * kRows, desc_add(dq, ks * 32), desc_add(dk, ks * 32), idS, ks > 0);
+        mma_commit(bars + kBarS + 8 * x);
       };
       auto issue_PV = [&](int x, int j) {
-        const uint64_t dp = sw128_desc(base + kOffP + x * kPTile, 16, 1024);
         const uint64_t dv = sw128_desc(base + kOffV + (j % kStages) * kTile, kTile, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + 2 * kRows + x * kD, desc_add(dp, (kk >> 2) * (kRows * 128) + (kk & 3) * 32),
-                   desc_add(dv, kk * 2048), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + kColO + x * kD, tmem + kColP + x * (kRows / 2) + 8 * kk,
+                      desc_add(dv, kk * 2048), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bars + kBarPV + 8 * x);
+      };
+      // tile x at key tile j: S_x(j+1) once S_x(j) is read, then P_x(j) V_j
+      auto step = [&](int x, int j, int n) -> bool {
+        if (j + 1 < n) {
+          const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
+          if (!mbar_wait(bars + kBarSF + 8 * x, j & 1, abort, status)) return false;
+          if (!mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status)) return false;
+          tc_fence_after();
+          issue_S(x, j + 1);
+        }
+        if (!mbar_wait(bars + kBarP + 8 * x, j & 1, abort, status)) return false;
+        if (!mbar_wait(bars + kBarV + 8 * (j % kStages), (j / kStages) & 1, abort, status)) return false;
+        tc_fence_after();
+        issue_PV(x, j);
+        return true;
       };
       bool ok = mbar_wait(bars + kBarQ, 0, abort, status) && mbar_wait(bars + kBarK, 0, abort, status);
       if (ok) {
         tc_fence_after();
         issue_S(0, 0);
-        mma_commit(bars + kBarS);
         issue_S(1, 0);
-        mma_commit(bars + kBarS + 8);
       }
       for (int j = 0; ok && j < nB; ++j) {
-        const int s = j % kStages, u = j / kStages;
-        const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
-        bool v_ready = false;
-        if (j < nA) {
-          if (!(ok = mbar_wait(bars + kBarP, j & 1, abort, status))) break;
-          if (!(ok = mbar_wait(bars + kBarV + 8 * s, u & 1, abort, status))) break;
-          v_ready = true;
-          tc_fence_after();
-          issue_PV(0, j);
-          if (j + 1 < nA) {
-            if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
-            issue_S(0, j + 1);
-            mma_commit(bars + kBarS);
-          } else {
-            mma_commit(bars + kBarO);
-          }
-        }
-        if (!(ok = mbar_wait(bars + kBarP + 8, j & 1, abort, status))) break;
-        if (!v_ready && !(ok = mbar_wait(bars + kBarV + 8 * s, u & 1, abort, status))) break;
-        tc_fence_after();
-        issue_PV(1, j);
-        if (j + 1 < nB) {
-          if (!(ok = mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status))) break;
-          issue_S(1, j + 1);
-          mma_commit(bars + kBarS + 8);
-        } else {
-          mma_commit(bars + kBarO + 8);
-        }
-        mma_commit(bars + kBarE + 8 * s);  // K_j and V_j free once these MMAs are done
+        if (j < nA && !(ok = step(0, j, nA))) break;
+        if (!(ok = step(1, j, nB))) break;
+        mma_commit(bars + kBarE + 8 * (j % kStages));  // K_j and V_j free once these MMAs are done
       }
       // Every MMA issued here has finished before TMEM is released.
       mma_commit(bars + kBarDrain);
@@ -205,19 +199,21 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int x = warp >> 3, h = (warp >> 2) & 1, wr = warp & 3;
     const int r = wr * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
-    const uint32_t tS = lane_base + x * kRows + 64 * h, tO = lane_base + 2 * kRows + x * kD + 32 * h;
+    const uint32_t tS = lane_base + x * kRows + 64 * h, tO = lane_base + kColO + x * kD + 32 * h;
+    const uint32_t tP = lane_base + kColP + x * (kRows / 2) + 32 * h;
     const int n = x ? nB : nA;
     const int qrow = q0 + x * kRows + r;
-    const uint32_t prow = base + kOffP + x * kPTile + h * (kRows * 128) + r * 128;
     float* red = reinterpret_cast<float*>(gbase + kOffRed);
     float* lsum = reinterpret_cast<float*>(gbase + kOffL);
     float m_ref = -INFINITY;
     float2 l2 = make_float2(0.f, 0.f);  // this half's row sum, two partial sums
     bool ok = true;
+    bool pv_seen = true;  // the previous P V product is known complete
     for (int j = 0; j < n; ++j) {
       ok = mbar_wait(bars + kBarS + 8 * x, j & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before TMEM access
       tc_fence_after();
+      pv_seen = j == 0;
       const bool diag = j == n - 1;
       // Keys after this query (only on the diagonal tile) are masked:
       // columns c of this half with 64 h + c > lim.
@@ -247,6 +243,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const float m_new = mx > m_ref + kRescale ? mx : m_ref;
       const float alpha = exp2f(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
       if (j > 0 && __any_sync(0xffffffffu, m_new != m_ref)) {
+        // O_x holds P V up to tile j-1: that product must be complete
+        ok = mbar_wait(bars + kBarPV + 8 * x, (j - 1) & 1, abort, status);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        pv_seen = true;
+        tc_fence_after();
         float o[32];
         tmem_ld32(tO, o);
         tmem_wait_ld();
@@ -258,11 +259,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       m_ref = m_new;
       l2.x *= alpha;
       l2.y *= alpha;
-      // P = 2^(s*sl2 - m_ref), row sum, bf16 P into this half's K-block.
-      // S is read from TMEM again rather than kept live across the exchange.
+      // P = 2^(s*sl2 - m_ref), row sum, bf16 P.  S is read from TMEM again
+      // rather than kept live across the exchange, then released.
       tmem_ld32(tS, v[0]);
       tmem_ld32(tS + 32, v[1]);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bars + kBarSF + 8 * x);
       if (diag) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -271,27 +274,26 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
       const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
+      uint32_t w[32];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
           t.x = ex2_approx(t.x);
           t.y = ex2_approx(t.y);
           l2 = fadd2(l2, t);
-          w[e >> 1] = pack_bf16x2(t.x, t.y);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = c * 4 + q;  // 16-byte chunk within this half's 128-byte row
-          const uint32_t dst = prow + ((ch ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(dst), "r"(w[4 * q]),
-                       "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
-                       : "memory");
+          w[c * 16 + (e >> 1)] = pack_bf16x2(t.x, t.y);
         }
       }
-      fence_proxy_async();
+      // P_x(j-1) must have been consumed before it is overwritten
+      if (!pv_seen) {
+        ok = mbar_wait(bars + kBarPV + 8 * x, (j - 1) & 1, abort, status);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      }
+      tc_fence_after();
+      tmem_st32u(tP, w);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + kBarP + 8 * x);
     }
@@ -301,7 +303,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_arrive(bars + kBarL + 8 * x);
       ok = mbar_wait(bars + kBarL + 8 * x, 0, abort, status);
     }
-    if (ok) ok = mbar_wait(bars + kBarO + 8 * x, 0, abort, status);
+    if (ok) ok = mbar_wait(bars + kBarPV + 8 * x, (n - 1) & 1, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
       const float l = lsum[(x * 2) * kRows + r] + lsum[(x * 2 + 1) * kRows + r];
       tc_fence_after();
