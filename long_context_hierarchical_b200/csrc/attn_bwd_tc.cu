@@ -202,7 +202,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                         const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ lse,
                         const float* __restrict__ Dv, bf16* __restrict__ dK, bf16* __restrict__ dV,
-                        int S, float sl2, float scale, unsigned int* __restrict__ status) {
+                        int S, float sl2, float scale, int tiles_on_y,
+                        unsigned int* __restrict__ status) {
   static_assert(C == kRows, "a dQ share has one TMEM lane per query of the chunk");
   using F = Cfg<C>;
   using L = KV<C>;
@@ -215,8 +216,9 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
   const float* vec = reinterpret_cast<const float*>(gbase + L::kOffVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // key tile; tile 0 sees the most query chunks
-  const int bh = blockIdx.y;
+  // key tile; tile 0 sees the most query chunks and is launched first
+  const int kt = tiles_on_y ? blockIdx.y : blockIdx.x;
+  const int bh = tiles_on_y ? blockIdx.x : blockIdx.y;
   const int k0 = kt * kRows;
   const int nq = (S - k0 + C - 1) / C;  // query chunks [k0 + C t, k0 + C t + C)
   const int row0 = bh * S;
@@ -473,7 +475,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
                       const float* __restrict__ lse, const float* __restrict__ Dv,
                       bf16* __restrict__ dQ, int S, int ntiles, float sl2, float scale,
-                      unsigned int* __restrict__ status) {
+                      int tiles_on_y, unsigned int* __restrict__ status) {
   using F = Cfg<C>;
   using L = QQ<C>;
   extern __shared__ uint8_t smem_raw[];
@@ -484,8 +486,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + L::kOffBar + L::kSlotAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = ntiles - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y;
+  const int qt = ntiles - 1 - (int)(tiles_on_y ? blockIdx.y : blockIdx.x);  // longest rows first
+  const int bh = tiles_on_y ? blockIdx.x : blockIdx.y;
   const int q0 = qt * kRows;
   const int kend = min(q0 + kRows, S);  // keys [0, kend) reach this tile
   const int nk = (kend + C - 1) / C;
@@ -673,7 +675,11 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   }
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float sl2 = 0.125f * kLog2e;
-  const dim3 grid(ntiles, (unsigned)BH);
+  // (problems, tiles): every problem's longest tile is launched before any
+  // shorter one, which keeps the tail of the grid short
+  const int ty = ntiles <= 65535 ? 1 : 0;
+  if (!ty && BH > 65535) return cudaErrorInvalidConfiguration;
+  const dim3 grid = ty ? dim3((unsigned)BH, ntiles) : dim3(ntiles, (unsigned)BH);
   if (dq_acc != nullptr) {
     const int64_t n = BH * S * kD;
     CUtensorMap accM;
@@ -682,7 +688,7 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
     if (e != cudaSuccess) return e;
     attn_bwd_dkdv_tc_kernel<C, true><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
         qC, kR, vR, gC, accM, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2,
-        0.125f, status);
+        0.125f, ty, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int64_t n8 = n / 8;
@@ -693,11 +699,11 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   }
   attn_bwd_dkdv_tc_kernel<C, false><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
       qC, kR, vR, gC, qC /* no dQ shares */, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV),
-      (int)S, sl2, 0.125f, status);
+      (int)S, sl2, 0.125f, ty, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dq_tc_kernel<C><<<grid, F::kThreads, QQ<C>::kSmemBytes, st>>>(
-      qR, kC, vC, gR, lse, D, static_cast<bf16*>(dQ), (int)S, ntiles, sl2, 0.125f, status);
+      qR, kC, vC, gR, lse, D, static_cast<bf16*>(dQ), (int)S, ntiles, sl2, 0.125f, ty, status);
   return cudaGetLastError();
 }
 

@@ -61,6 +61,24 @@ constexpr uint32_t kOffL = kOffRed + 2 * 2 * 2 * kRows * 4;
 constexpr uint32_t kSmemBytes = kOffL + 2 * 2 * kRows * 4 + 1024;  // + alignment slack
 static_assert(kSlotAbort + 4 <= 256, "barrier area");
 
+// P = 2^(s * sl2 - m) for this thread's 64 scores, their sum into l2, and P
+// as bf16 pairs.
+__device__ __forceinline__ void exp_row(const float (&v)[2][32], float sl2, float m, float2& l2,
+                                        uint32_t (&w)[32]) {
+  const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
+      t.x = ex2_approx(t.x);
+      t.y = ex2_approx(t.y);
+      l2 = fadd2(l2, t);
+      w[c * 16 + (e >> 1)] = pack_bf16x2(t.x, t.y);
+    }
+  }
+}
+
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   // Bounded wait that ignores the abort flag (used to drain own copies).
   const long long t0 = clock64();
@@ -74,7 +92,7 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ O,
-                   float* __restrict__ lse, int S, int npairs, float sl2,
+                   float* __restrict__ lse, int S, int npairs, float sl2, int tiles_on_y,
                    unsigned int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -84,8 +102,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + kOffBar + kSlotAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = npairs - 1 - (int)blockIdx.x;  // longest rows first
-  const int bh = blockIdx.y;
+  const int pair = npairs - 1 - (int)(tiles_on_y ? blockIdx.y : blockIdx.x);  // longest rows first
+  const int bh = tiles_on_y ? blockIdx.x : blockIdx.y;
   const int q0 = pair * 2 * kRows;
   const int nA = 2 * pair + 1, nB = 2 * pair + 2;  // key tiles of tile A / tile B
   const int row0 = bh * S;                          // first row of this head in the maps
@@ -273,19 +291,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           if (32 + e > lim) v[1][e] = -INFINITY;
         }
       }
-      const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_ref, -m_ref);
       uint32_t w[32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
-          t.x = ex2_approx(t.x);
-          t.y = ex2_approx(t.y);
-          l2 = fadd2(l2, t);
-          w[c * 16 + (e >> 1)] = pack_bf16x2(t.x, t.y);
-        }
-      }
+      exp_row(v, sl2, m_ref, l2, w);
       // P_x(j-1) must have been consumed before it is overwritten
       if (!pv_seen) {
         ok = mbar_wait(bars + kBarPV + 8 * x, (j - 1) & 1, abort, status);
@@ -391,8 +398,12 @@ cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   }
   const int npairs = (int)((S + 2 * kRows - 1) / (2 * kRows));
   const float sl2 = 0.125f * 1.4426950408889634f;
-  attn_fwd_tc_kernel<<<dim3(npairs, (unsigned)BH), kThreads, kSmemBytes, st>>>(
-      mq, mk, mv, static_cast<bf16*>(O), lse, (int)S, npairs, sl2, status);
+  // (problems, tile pairs): every problem's longest pair is launched first
+  const int ty = npairs <= 65535 ? 1 : 0;
+  if (!ty && BH > 65535) return cudaErrorInvalidConfiguration;
+  const dim3 grid = ty ? dim3((unsigned)BH, npairs) : dim3(npairs, (unsigned)BH);
+  attn_fwd_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, static_cast<bf16*>(O), lse, (int)S,
+                                                        npairs, sl2, ty, status);
   return cudaGetLastError();
 }
 
