@@ -145,6 +145,23 @@ __device__ __forceinline__ void gemm_acc_ts(uint32_t d, uint32_t a_tmem, uint32_
     mma_bf16_ts(d, a_tmem + 8 * kk, desc_add(db, kk * 2048), idesc, (acc || kk > 0) ? 1u : 0u);
 }
 
+// Byte offset of row r, column 0 of a K=16 slice (no swizzle).
+__device__ __forceinline__ uint32_t slice_off(int r) { return (r >> 3) * 256 + (r & 7) * 16; }
+// Descriptor of a K=16 slice: no swizzle, K-direction core matrices 128
+// bytes apart, 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t slice_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(256 >> 4) << 32) |
+         (1ull << 46);
+}
+// v split into three bf16 parts a + b + c (each the rounding of what the
+// previous ones leave), stored in columns 0-2 of a slice row.
+__device__ __forceinline__ void store_split3(uint8_t* row, float v) {
+  const float a = __bfloat162float(__float2bfloat16_rn(v));
+  const float b = __bfloat162float(__float2bfloat16_rn(v - a));
+  *reinterpret_cast<uint32_t*>(row) = pack_bf16x2(a, b);
+  *reinterpret_cast<__nv_bfloat16*>(row + 4) = __float2bfloat16_rn((v - a) - b);
+}
+
 // ===========================================================================
 // dK, dV (and, fused, the dQ shares)
 // ===========================================================================
@@ -154,7 +171,17 @@ __device__ __forceinline__ void gemm_acc_ts(uint32_t d, uint32_t a_tmem, uint32_
 // Shared memory: K, V tiles; kStages x (Q chunk, dO chunk); dS^T (K-major,
 // also read MN-major by the dQ product); the dQ staging area: four boxes of
 // 128 rows x 16 fp32 (64-byte swizzle), one per element-wise group, each
-// reduced into the fp32 accumulator by one TMA reduce-add.
+// reduced into the fp32 accumulator by one TMA reduce-add; and the K=16
+// slices that fold the per-query terms into the MMAs (below).
+//
+// The per-query terms lse and D enter through one extra K=16 step of the
+// S^T and dP^T products instead of per-column loads in the element-wise
+// loop: a constant slice with -1 in columns 0-2 for every key row times a
+// per-chunk slice holding, for each query, a three-part bf16 split of
+// lse * log2(e) / (scale * log2(e)) (for S^T) or of D (for dP^T), zeros
+// elsewhere.  So S^T holds s - lse / scale and dP^T holds dP - D, to about
+// 2^-25 of the folded term.  The slices are K-major without swizzle:
+// element (r, k) at (r / 8) * 256 + (k / 8) * 128 + (r % 8) * 16 + (k % 8) * 2.
 template <int C>
 struct KV {
   using F = Cfg<C>;
@@ -164,8 +191,11 @@ struct KV {
   static constexpr uint32_t kOffDST = kOffG + F::kStages * F::kTileC;  // dS^T (128 x C)
   static constexpr uint32_t kOffStage = kOffDST + F::kWide;            // 4 x 8 KB dQ boxes
   static constexpr uint32_t kStageBox = kRows * 16 * 4;
-  static constexpr uint32_t kOffVec = kOffStage + 4 * kStageBox;       // kStages x (C lse2 + C D)
-  static constexpr uint32_t kOffBar = kOffVec + F::kStages * 2 * C * 4;
+  static constexpr uint32_t kSlice = kRows * 16 * 2;                   // 4 KB K=16 slice
+  static constexpr uint32_t kOffNeg = kOffStage + 4 * kStageBox;       // the -1 slice
+  static constexpr uint32_t kOffLx = kOffNeg + kSlice;                 // kStages lse slices
+  static constexpr uint32_t kOffDx = kOffLx + F::kStages * kSlice;     // kStages D slices
+  static constexpr uint32_t kOffBar = kOffDx + F::kStages * kSlice;
   static constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * F::kStages,
                             kBarSP = kBarEmpty + 8 * F::kStages, kBarPDS = kBarSP + 8,
                             kBarAcc = kBarPDS + 8, kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8,
@@ -213,7 +243,6 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
   uint8_t* gbase = smem_raw + (base - raw);
   const uint32_t bars = base + L::kOffBar;
   volatile int* abort = reinterpret_cast<volatile int*>(gbase + L::kOffBar + L::kSlotAbort);
-  const float* vec = reinterpret_cast<const float*>(gbase + L::kOffVec);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // key tile; tile 0 sees the most query chunks and is launched first
@@ -240,6 +269,15 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     *abort = 0;
     fence_mbar_init();
   }
+  // the K=16 slices: zero, then -1 in columns 0-2 of the constant one
+  for (uint32_t i = threadIdx.x; i < (1 + 2 * F::kStages) * L::kSlice / 16; i += blockDim.x)
+    *reinterpret_cast<uint4*>(gbase + L::kOffNeg + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if (threadIdx.x < kRows) {
+    *reinterpret_cast<uint32_t*>(gbase + L::kOffNeg + slice_off(threadIdx.x)) = 0xBF80BF80u;  // -1, -1
+    *reinterpret_cast<uint16_t*>(gbase + L::kOffNeg + slice_off(threadIdx.x) + 4) = 0xBF80u;  // -1
+  }
+  fence_proxy_async();
   if (warp == F::kMmaWarp) tmem_alloc(bars + L::kSlotTmem, L::kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -254,6 +292,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       tma_load_2d(base + L::kOffK, &tmK, 0, row0 + k0, bars + L::kBarKV);
       tma_load_2d(base + L::kOffV, &tmV, 0, row0 + k0, bars + L::kBarKV);
     }
+    const float inv_scale = 1.f / scale;  // lse * log2(e) / (scale * log2(e))
     for (int t = 0; t < nq; ++t) {
       const int s = t % F::kStages, u = t / F::kStages;
       bool go = true;
@@ -265,14 +304,15 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         tma_load_2d(base + L::kOffQ + s * F::kTileC, &tmQ, 0, row0 + q0, bars + L::kBarFull + 8 * s);
         tma_load_2d(base + L::kOffG + s * F::kTileC, &tmG, 0, row0 + q0, bars + L::kBarFull + 8 * s);
       }
-      float* dst = reinterpret_cast<float*>(gbase + L::kOffVec + s * 2 * C * 4);
 #pragma unroll
       for (int e = 0; e < C / 32; ++e) {
         const int q = 32 * e + lane;
         const bool in = q0 + q < S;
-        dst[q] = in ? lse[row0 + q0 + q] * kLog2e : 0.f;
-        dst[C + q] = in ? Dv[row0 + q0 + q] : 0.f;
+        const uint32_t off = slice_off(q);
+        store_split3(gbase + L::kOffLx + s * L::kSlice + off, in ? lse[row0 + q0 + q] * inv_scale : 0.f);
+        store_split3(gbase + L::kOffDx + s * L::kSlice + off, in ? Dv[row0 + q0 + q] : 0.f);
       }
+      fence_proxy_async();  // the slices are read by the tensor core
       mbar_arrive(bars + L::kBarFull + 8 * s);
       issued = t + 1;
     }
@@ -287,11 +327,17 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       constexpr uint32_t idS = idesc_bf16(kRows, C, false);
       bool ok = mbar_wait(bars + L::kBarKV, 0, abort, status) &&
                 mbar_wait(bars + L::kBarFull, 0, abort, status);
+      // S^T - lse / scale = K Q^T - lse slice, dP^T - D = V dO^T - D slice
+      auto issue_sp = [&](int s1) {
+        gemm_sq(tmem, base + L::kOffK, base + L::kOffQ + s1 * F::kTileC, idS);
+        mma_bf16(tmem, slice_desc(base + L::kOffNeg), slice_desc(base + L::kOffLx + s1 * L::kSlice), idS, 1u);
+        gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG + s1 * F::kTileC, idS);
+        mma_bf16(tmem + C, slice_desc(base + L::kOffNeg), slice_desc(base + L::kOffDx + s1 * L::kSlice), idS, 1u);
+        mma_commit(bars + L::kBarSP);
+      };
       if (ok) {
         tc_fence_after();
-        gemm_sq(tmem, base + L::kOffK, base + L::kOffQ, idS);      // S^T = K Q^T
-        gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG, idS);  // dP^T = V dO^T
-        mma_commit(bars + L::kBarSP);
+        issue_sp(0);
       }
       // dQ share j: issued as step j's last MMA, staged by the element-wise
       // warps after step j+1's P/dS hand-off (QD), reduced from here into
@@ -309,9 +355,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         if (t + 1 < nq) {
           const int s1 = (t + 1) % F::kStages, u1 = (t + 1) / F::kStages;
           if (!(ok = mbar_wait(bars + L::kBarFull + 8 * s1, u1 & 1, abort, status))) break;
-          gemm_sq(tmem, base + L::kOffK, base + L::kOffQ + s1 * F::kTileC, idS);
-          gemm_sq(tmem + C, base + L::kOffV, base + L::kOffG + s1 * F::kTileC, idS);
-          mma_commit(bars + L::kBarSP);
+          issue_sp(s1);
         }
         if constexpr (kFused) {
           if (t >= 2) {  // share t-2's reduce has read the boxes
@@ -374,8 +418,6 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       const int q0 = k0 + t * C;
       // visible: key <= query < S
       const bool edge = (q0 < k0 + kRows) || (q0 + C > S);
-      const float* l2 = vec + s * 2 * C + col0;
-      const float* dd = l2 + C;
       float st[32], dp[32];
       tmem_ld32(lane_base + col0, st);
       tmem_ld32(lane_base + C + col0, dp);
@@ -385,10 +427,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
       uint32_t wp[16], wd[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
-        const float4 lv = *reinterpret_cast<const float4*>(l2 + e);
-        const float4 dv = *reinterpret_cast<const float4*>(dd + e);
-        float2 x0 = ffma2(make_float2(st[e], st[e + 1]), sc2, make_float2(-lv.x, -lv.y));
-        float2 x1 = ffma2(make_float2(st[e + 2], st[e + 3]), sc2, make_float2(-lv.z, -lv.w));
+        const float2 x0 = fmul2(make_float2(st[e], st[e + 1]), sc2);
+        const float2 x1 = fmul2(make_float2(st[e + 2], st[e + 3]), sc2);
         float p[4] = {ex2_approx(x0.x), ex2_approx(x0.y), ex2_approx(x1.x), ex2_approx(x1.y)};
         if (edge) {
 #pragma unroll
@@ -399,8 +439,10 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         }
         wp[e >> 1] = pack_bf16x2(p[0], p[1]);
         wp[(e >> 1) + 1] = pack_bf16x2(p[2], p[3]);
-        wd[e >> 1] = pack_bf16x2(p[0] * (dp[e] - dv.x), p[1] * (dp[e + 1] - dv.y));
-        wd[(e >> 1) + 1] = pack_bf16x2(p[2] * (dp[e + 2] - dv.z), p[3] * (dp[e + 3] - dv.w));
+        const float2 d0 = fmul2(make_float2(p[0], p[1]), make_float2(dp[e], dp[e + 1]));
+        const float2 d1 = fmul2(make_float2(p[2], p[3]), make_float2(dp[e + 2], dp[e + 3]));
+        wd[e >> 1] = pack_bf16x2(d0.x, d0.y);
+        wd[(e >> 1) + 1] = pack_bf16x2(d1.x, d1.y);
       }
       // the previous step's P^T / dS^T (and dQ share) must be consumed before
       // they are overwritten

@@ -186,10 +186,13 @@ def test_attention_backward(case, deterministic):
 
 
 def test_attention_backward_schedules_agree(case):
-    """The fused schedule (dQ shares added with fp32 atomics) and the
+    """The fused schedule (dQ shares reduce-added in fp32) and the
     deterministic two-kernel one: dK, dV from the same kernel code are
-    bit-identical, dQ differs only by the order of its fp32 sum; the
-    deterministic schedule repeats bit for bit."""
+    bit-identical; dQ agrees to the rounding of its terms (the fused kernel
+    forms dS with lse and D folded into its MMAs, the dq kernel subtracts
+    them in fp32, so a dS element may round to the neighbouring bf16 value,
+    and the fp32 sums run in different orders); the deterministic schedule
+    repeats bit for bit."""
     c = case
     lh, dt = c["lh"], c["dt"]
     Qg, Kg, Vg, Og = (_t(stack(c["ctxs"], k), dt) for k in ("Qg", "Kg", "Vg", "Og"))
@@ -205,11 +208,13 @@ def test_attention_backward_schedules_agree(case):
         assert torch.equal(a, b)
     assert torch.equal(fused[1], det[0][1]) and torch.equal(fused[2], det[0][2])
     a, b = np64(fused[0]), np64(det[0][0])
-    # both are fp32 sums of the same shares rounded once: at most one rounding
-    # step of the output type apart, plus fp32 reordering under cancellation
+    # one rounding step of the output, plus one bf16 rounding of each term
+    # (dS differently rounded) within the term bound tq = sum |dS| |K| (and more)
     step = 2.0 ** -7 if dt == torch.bfloat16 else 2.0 ** -22
     tq = c["terms"]["dQg"]
-    assert np.all(np.abs(a - b) <= step * np.abs(b) + 2.0 ** -14 * tq + 1e-30), "dQg fused vs deterministic"
+    err = np.abs(a - b)
+    bad = err > step * np.abs(b) + step / 2 * tq + 1e-30
+    assert not bad.any(), f"dQg fused vs deterministic: {int(bad.sum())} elements, max {err.max():.3e}"
 
 
 def test_gather_backward(case):
