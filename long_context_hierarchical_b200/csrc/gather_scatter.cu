@@ -10,9 +10,9 @@
 // Backward ("梯度流": dL -> scatter -> attention -> gather): the adjoints of
 // those two maps, plus the softmax-backward row term D.
 //
-// All four kernels are "one 8-lane group per row": lane c of a group moves
-// channels [8c, 8c+8) with 16-byte accesses, so a warp touches 4 whole rows
-// per instruction.  The scatter and gather-backward kernels are
+// The gather and scatter-backward kernels give each row to 8 lanes: lane c
+// moves channels [8c, 8c+8) with 16-byte accesses, so a warp touches 4 whole
+// rows per instruction (the scatter and gather-backward split is below).  The scatter and gather-backward kernels are
 // token-centric and sum in a fixed (ascending-level) order: no atomics, and
 // the result does not depend on scheduling.
 #include "host.h"
@@ -87,13 +87,19 @@ __device__ __forceinline__ void store_stream<float>(float* p, const float (&x)[8
 
 // p = 2^LOGP and L are template parameters, the head comes from blockIdx.y
 // and indices inside a head are 32-bit, so the per-token index arithmetic is
-// a handful of shifts and adds.
+// a handful of shifts and adds.  The token-centric kernels (scatter, gather
+// backward) give each row to 4 lanes, lane c moving chunks c and c + 4, so
+// the per-token index work is shared by fewer lanes (these kernels are
+// instruction-bound with 8 lanes per row) while every store instruction
+// still covers whole 32-byte sectors.
+constexpr int kRowsPerBlock4 = kThreads / 4;
+
 template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
-  const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
-  const int c = threadIdx.x & 7;
+  const int t = blockIdx.x * kRowsPerBlock4 + (threadIdx.x >> 2);
+  const int c = threadIdx.x & 3;
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
@@ -105,19 +111,26 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
     const int i = ((t + 1) >> (LOGP * l)) - 1;
     slot[l] = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
   }
-  float acc[8];
+  float a0[8], a1[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) a0[e] = a1[e] = 0.f;
 #pragma unroll
   for (int l = 0; l < L; ++l) {  // ascending level
     if ((unsigned)slot[l] < (unsigned)S) {
-      float x[8];
-      Vec8<T>::load(og + (int64_t)slot[l] * kD, x);
+      float x0[8], x1[8];
+      const T* src = og + (int64_t)slot[l] * kD;
+      Vec8<T>::load(src, x0);
+      Vec8<T>::load(src + 32, x1);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += x[e];
+      for (int e = 0; e < 8; ++e) {
+        a0[e] += x0[e];
+        a1[e] += x1[e];
+      }
     }
   }
-  store_stream<T>(O + (bh * g.N + t) * kD + c * 8, acc);
+  T* dst = O + (bh * g.N + t) * kD + c * 8;
+  store_stream<T>(dst, a0);
+  store_stream<T>(dst + 32, a1);
 }
 
 template <typename T, int LOGP, int L>
@@ -178,8 +191,8 @@ __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
                   T* __restrict__ dQ, T* __restrict__ dK, T* __restrict__ dV) {
-  const int t = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
-  const int c = threadIdx.x & 7;
+  const int t = blockIdx.x * kRowsPerBlock4 + (threadIdx.x >> 2);
+  const int c = threadIdx.x & 3;
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
@@ -193,24 +206,31 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
-    float acc[8];
+    float a0[8], a1[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) a0[e] = a1[e] = 0.f;
 #pragma unroll
     for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
       if ((unsigned)slot[l] < (unsigned)S) {
-        float x[8];
-        Vec8<T>::load(src[w] + base + (int64_t)slot[l] * kD, x);
+        float x0[8], x1[8];
+        const T* p = src[w] + base + (int64_t)slot[l] * kD;
+        Vec8<T>::load(p, x0);
+        Vec8<T>::load(p + 32, x1);
         const float wgt = 1.f / (float)(1 << (LOGP * l));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(x[e], wgt, acc[e]);
+        for (int e = 0; e < 8; ++e) {
+          a0[e] = fmaf(x0[e], wgt, a0[e]);
+          a1[e] = fmaf(x1[e], wgt, a1[e]);
+        }
       }
     }
-    store_stream<T>(dst[w] + out, acc);
+    store_stream<T>(dst[w] + out, a0);
+    store_stream<T>(dst[w] + out + 32, a1);
   }
 }
 
 unsigned blocks_for(int64_t rows) { return (unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock); }
+unsigned blocks_for4(int64_t rows) { return (unsigned)((rows + kRowsPerBlock4 - 1) / kRowsPerBlock4); }
 
 }  // namespace
 
@@ -257,7 +277,7 @@ void with_levels(const Geo& g, F&& f) {
 
 template <typename T>
 void scatter_t(const Geo& g, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
-  const dim3 grid((unsigned)((g.N + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
     scatter_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
   });
@@ -292,7 +312,7 @@ cudaError_t launch_scatter_bwd(const lh_plan& plan, const void* dO, const void* 
 template <typename T>
 void gather_bwd_t(const Geo& g, const void* dQg, const void* dKg, const void* dVg,
                   const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
-  const dim3 grid((unsigned)((g.N + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
     gather_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(
         g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
