@@ -88,18 +88,20 @@ __device__ __forceinline__ void store_stream<float>(float* p, const float (&x)[8
 // p = 2^LOGP and L are template parameters, the head comes from blockIdx.y
 // and indices inside a head are 32-bit, so the per-token index arithmetic is
 // a handful of shifts and adds.  The token-centric kernels (scatter, gather
-// backward) give each row to 4 lanes, lane c moving chunks c and c + 4, so
-// the per-token index work is shared by fewer lanes (these kernels are
+// backward) give each row to R lanes, lane c moving chunks c, c + R, ...,
+// so the per-token index work is shared by fewer lanes (these kernels are
 // instruction-bound with 8 lanes per row) while every store instruction
 // still covers whole 32-byte sectors.
-constexpr int kRowsPerBlock4 = kThreads / 4;
+constexpr int kLanesPerRow = 4;
+constexpr int kChunks = 8 / kLanesPerRow;  // 8-element chunks per lane
+constexpr int kRowsPerBlock4 = kThreads / kLanesPerRow;
 
 template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
-  const int t = blockIdx.x * kRowsPerBlock4 + (threadIdx.x >> 2);
-  const int c = threadIdx.x & 3;
+  const int t = blockIdx.x * kRowsPerBlock4 + (int)(threadIdx.x / kLanesPerRow);
+  const int c = threadIdx.x % kLanesPerRow;
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
@@ -111,26 +113,27 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
     const int i = ((t + 1) >> (LOGP * l)) - 1;
     slot[l] = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
   }
-  float a0[8], a1[8];
+  float a[kChunks][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) a0[e] = a1[e] = 0.f;
+  for (int k = 0; k < kChunks; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
   for (int l = 0; l < L; ++l) {  // ascending level
     if ((unsigned)slot[l] < (unsigned)S) {
-      float x0[8], x1[8];
       const T* src = og + (int64_t)slot[l] * kD;
-      Vec8<T>::load(src, x0);
-      Vec8<T>::load(src + 32, x1);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        a0[e] += x0[e];
-        a1[e] += x1[e];
+      for (int k = 0; k < kChunks; ++k) {
+        float x[8];
+        Vec8<T>::load(src + 8 * kLanesPerRow * k, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[k][e] += x[e];
       }
     }
   }
   T* dst = O + (bh * g.N + t) * kD + c * 8;
-  store_stream<T>(dst, a0);
-  store_stream<T>(dst + 32, a1);
+#pragma unroll
+  for (int k = 0; k < kChunks; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
 }
 
 template <typename T, int LOGP, int L>
@@ -191,8 +194,8 @@ __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
                   T* __restrict__ dQ, T* __restrict__ dK, T* __restrict__ dV) {
-  const int t = blockIdx.x * kRowsPerBlock4 + (threadIdx.x >> 2);
-  const int c = threadIdx.x & 3;
+  const int t = blockIdx.x * kRowsPerBlock4 + (int)(threadIdx.x / kLanesPerRow);
+  const int c = threadIdx.x % kLanesPerRow;
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
@@ -206,26 +209,27 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
-    float a0[8], a1[8];
+    float a[kChunks][8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) a0[e] = a1[e] = 0.f;
+    for (int k = 0; k < kChunks; ++k)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
     for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
       if ((unsigned)slot[l] < (unsigned)S) {
-        float x0[8], x1[8];
         const T* p = src[w] + base + (int64_t)slot[l] * kD;
-        Vec8<T>::load(p, x0);
-        Vec8<T>::load(p + 32, x1);
         const float wgt = 1.f / (float)(1 << (LOGP * l));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          a0[e] = fmaf(x0[e], wgt, a0[e]);
-          a1[e] = fmaf(x1[e], wgt, a1[e]);
+        for (int k = 0; k < kChunks; ++k) {
+          float x[8];
+          Vec8<T>::load(p + 8 * kLanesPerRow * k, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[k][e] = fmaf(x[e], wgt, a[k][e]);
         }
       }
     }
-    store_stream<T>(dst[w] + out, a0);
-    store_stream<T>(dst[w] + out + 32, a1);
+#pragma unroll
+    for (int k = 0; k < kChunks; ++k) store_stream<T>(dst[w] + out + 8 * kLanesPerRow * k, a[k]);
   }
 }
 

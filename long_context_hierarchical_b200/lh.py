@@ -13,7 +13,9 @@ from dataclasses import dataclass
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "liblh.so")
+# LH_LIBRARY selects another build of the library (for example a variant
+# compiled with different tile constants); the default is the in-tree one.
+LIB_PATH = os.environ.get("LH_LIBRARY") or os.path.join(HERE, "liblh.so")
 
 LH_OK, LH_ERR_INVALID_ARG, LH_ERR_UNSUPPORTED, LH_ERR_WORKSPACE, LH_ERR_CUDA, LH_ERR_TIMEOUT = range(6)
 LH_F32, LH_BF16 = 0, 1
