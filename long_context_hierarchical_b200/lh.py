@@ -359,6 +359,76 @@ def backward(pl: Plan, dO, ctx: Context, dQ=None, dK=None, dV=None, ws: Workspac
     return dQ, dK, dV
 
 
+class HostPipeline:
+    """Forward and backward of one layer per step on host (pinned) tensors.
+
+    Each step copies Q, K, V, dO to the device, runs lh_forward and
+    lh_backward, and copies O, dQ, dK, dV back.  Two device buffer sets and
+    three streams let the copy-in of step i+1 and the copy-out of step i-1
+    run while the kernels of step i do (PCIe is full duplex; the kernels use
+    only the compute stream).  ``step`` enqueues and returns at once;
+    ``synchronize`` waits for every enqueued step.  The host tensors passed to
+    a step must stay untouched until it has completed.
+    """
+
+    def __init__(self, pl: Plan, device):
+        c = pl.raw.c
+        shape = (c.B, c.H, c.N, c.d)
+        self.pl = pl
+        self.inputs = [[torch.empty(shape, dtype=pl.dtype, device=device) for _ in range(4)]
+                       for _ in range(2)]
+        self.outputs = [[torch.empty(shape, dtype=pl.dtype, device=device) for _ in range(4)]
+                        for _ in range(2)]
+        self.ctx = Context(pl, device)
+        self.ws = Workspace(pl, device)
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(device) for _ in range(3))
+        self.copied_in = [torch.cuda.Event() for _ in range(2)]
+        self.done = [torch.cuda.Event() for _ in range(2)]
+        self.copied_out = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+        self.n = 0
+
+    def step(self, host_inputs, host_outputs):
+        """host_inputs: (Q, K, V, dO); host_outputs: (O, dQ, dK, dV); pinned, [B,H,N,d]."""
+        b = self.n % 2
+        self.n += 1
+        dev_in, dev_out = self.inputs[b], self.outputs[b]
+        if self.used[b]:  # this buffer set's previous step has read its inputs
+            self.s_in.wait_event(self.done[b])
+        with torch.cuda.stream(self.s_in):
+            for d, h in zip(dev_in, host_inputs):
+                d.copy_(h, non_blocking=True)
+            self.copied_in[b].record(self.s_in)
+        self.s_run.wait_event(self.copied_in[b])
+        if self.used[b]:  # and its outputs have left the device
+            self.s_run.wait_event(self.copied_out[b])
+        Q, K, V, dO = dev_in
+        O, dQ, dK, dV = dev_out
+        forward(self.pl, Q, K, V, O, self.ctx, self.ws, stream=self.s_run)
+        backward(self.pl, dO, self.ctx, dQ, dK, dV, self.ws, stream=self.s_run)
+        self.done[b].record(self.s_run)
+        self.s_out.wait_event(self.done[b])
+        with torch.cuda.stream(self.s_out):
+            for h, d in zip(host_outputs, dev_out):
+                h.copy_(d, non_blocking=True)
+            self.copied_out[b].record(self.s_out)
+        self.used[b] = True
+
+    def wait_on(self, event):
+        """Make every stream of the pipeline wait for `event` (e.g. a start marker)."""
+        for st in (self.s_in, self.s_run, self.s_out):
+            st.wait_event(event)
+
+    def record_end(self, stream):
+        """Make `stream` wait for everything enqueued so far."""
+        for ev in self.copied_in + self.done + self.copied_out:
+            stream.wait_event(ev)
+
+    def synchronize(self):
+        for st in (self.s_in, self.s_run, self.s_out):
+            st.synchronize()
+
+
 def set_deterministic(on: bool):
     """Process-wide: bit-reproducible bf16 attention backward (two kernels, no
     atomics) for lh_attn_bwd / lh_backward calls enqueued afterwards."""

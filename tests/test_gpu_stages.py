@@ -257,6 +257,34 @@ def test_whole_layer(case):
     lh.device_status()
 
 
+def test_host_pipeline_matches_device_calls():
+    """lh.HostPipeline (host tensors, copies overlapping the kernels, two device
+    buffer sets) returns what lh.forward / lh.backward return on the device, for
+    every step of a sequence with different inputs (deterministic mode: bit for bit)."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k = 1, 4, 2048, 4, 3, 32
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16")
+    steps = [make_inputs(B, H, N, 64, "bf16", seed=20 + i) for i in range(3)]
+    lh.set_deterministic(True)
+    try:
+        pipe = lh.HostPipeline(pl, "cuda")
+        host_in = [tuple(x.pin_memory() for x in s) for s in steps]
+        host_out = [tuple(torch.empty_like(x).pin_memory() for x in s) for s in steps]
+        for hi, ho in zip(host_in, host_out):
+            pipe.step(hi, ho)
+        pipe.synchronize()
+        for (Q, K, V, dO), ho in zip(steps, host_out):
+            Qd, Kd, Vd, dOd = (x.cuda() for x in (Q, K, V, dO))
+            O, ctx = lh.forward(pl, Qd, Kd, Vd)
+            grads = lh.backward(pl, dOd, ctx)
+            torch.cuda.synchronize()
+            for got, exp in zip(ho, (O, *grads)):
+                assert torch.equal(got, exp.cpu())
+    finally:
+        lh.set_deterministic(False)
+    lh.device_status()
+
+
 def test_dense_fixed_point_matches_attention():
     """L = 1: the layer is plain causal attention on Q, K, V (skill card, 选择-注意力解耦)."""
     from long_context_hierarchical_b200 import lh
