@@ -3,20 +3,21 @@
 // stage 3: a standard S x S causal mask; gist.science 2.C).
 //
 // One CTA owns 256 query rows as two 128-row tiles A and B and walks the key
-// tiles (128 keys) up to its diagonal.  Warp roles (576 threads):
-//   warps 0-7  softmax of tile A, warps 8-15 softmax of tile B, each tile's
-//              eight warps as two groups on column halves [0,64), [64,128):
-//              thread r of a group owns query row r of its tile (TMEM lane
-//              r), so a row's max and sum need no shuffles, only one
-//              exchange of the two halves' maxima through shared memory;
-//   warp 16    TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
-//   warp 17    TMEM allocation and the single MMA-issuing thread.
+// tiles (128 keys) up to its diagonal.  Warp roles (320 threads):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
+//              tile's four warps owns query row r (TMEM lane r) and all 128
+//              columns of it, so a row's max and sum stay in one thread;
+//   warp 8     TMA producer: Q tiles once, then K/V tiles into a 3-stage ring;
+//   warp 9     TMEM allocation and the single MMA-issuing thread.
+// Each SM sub-partition runs one softmax warp of each tile (warp w sits on
+// sub-partition w % 4), so one tile's exponentials fill the special-function
+// unit while the other tile waits for its MMAs.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,320), O_B [320,384)
 // fp32; P_A [384,448), P_B [448,512) as bf16 pairs.  Per key tile j the MMA
 // thread issues S_X = Q_X K_j^T (M=128, N=128, 4 x K=16) and, once softmax X
 // has written P_X into TMEM, O_X += P_X V_j (A from TMEM, V read MN-major).
-// Softmax X releases S_X as soon as it has read it (before its
-// exponentials), so S_X for tile j+1 is computed while it works on tile j;
+// Softmax X releases S_X as soon as it has loaded it into registers, so S_X
+// for tile j+1 is computed while it works on tile j;
 // it waits for the previous P V product only before overwriting P_X (or
 // rescaling O_X).  O is rescaled in TMEM only when a row maximum grows by
 // more than 2^8 (the reference maximum otherwise stays, so P <= 256).
@@ -38,7 +39,7 @@ using namespace tc;
 constexpr int kRows = 128;                    // query rows per tile, keys per tile
 constexpr int kStages = 3;
 constexpr uint32_t kTile = kRows * kD * 2;    // 16 KB: 128 rows x 128 B
-constexpr int kLoadWarp = 16, kMmaWarp = 17;
+constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescale = 8.0f;              // log2 units
@@ -52,31 +53,19 @@ constexpr uint32_t kOffBar = kOffV + kStages * kTile;
 // per tile x (8 bytes apart): S ready, S freed, P written, P V done
 constexpr uint32_t kBarQ = 0, kBarK = 8, kBarV = kBarK + 8 * kStages, kBarE = kBarV + 8 * kStages,
                    kBarS = kBarE + 8 * kStages, kBarSF = kBarS + 16, kBarP = kBarSF + 16,
-                   kBarPV = kBarP + 16, kBarDrain = kBarPV + 16, kBarRed = kBarDrain + 8,
-                   kBarL = kBarRed + 32, kSlotTmem = kBarL + 16, kSlotAbort = kSlotTmem + 4;
-// Row-max exchange between the two column halves: [parity][tile][half][row];
-// then the row-sum exchange: [tile][half][row].
-constexpr uint32_t kOffRed = kOffBar + 256;
-constexpr uint32_t kOffL = kOffRed + 2 * 2 * 2 * kRows * 4;
-constexpr uint32_t kSmemBytes = kOffL + 2 * 2 * kRows * 4 + 1024;  // + alignment slack
+                   kBarPV = kBarP + 16, kBarDrain = kBarPV + 16, kSlotTmem = kBarDrain + 8,
+                   kSlotAbort = kSlotTmem + 4;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 static_assert(kSlotAbort + 4 <= 256, "barrier area");
 
-// P = 2^(s * sl2 - m) for this thread's 64 scores, their sum into l2, and P
-// as bf16 pairs.
-__device__ __forceinline__ void exp_row(const float (&v)[2][32], float sl2, float m, float2& l2,
-                                        uint32_t (&w)[32]) {
-  const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m, -m);
+// Maximum of this thread's 128 scores, as four independent chains.
+__device__ __forceinline__ float row_max(const float (&v)[4][32]) {
+  float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < 4; ++c)
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
-      t.x = ex2_approx(t.x);
-      t.y = ex2_approx(t.y);
-      l2 = fadd2(l2, t);
-      w[c * 16 + (e >> 1)] = pack_bf16x2(t.x, t.y);
-    }
-  }
+    for (int e = 0; e < 32; e += 2) pm[c] = fmax3f(pm[c], v[c][e], v[c][e + 1]);
+  return fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
 }
 
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
@@ -87,9 +76,9 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-// 18 warps: five of them share one SM sub-partition's 16K registers, so 96
+// 10 warps: three of them share one SM sub-partition's 16K registers, so 168
 // registers per thread is the most a launch can have.
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(168)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, bf16* __restrict__ O,
                    float* __restrict__ lse, int S, int npairs, float sl2, int tiles_on_y,
@@ -117,12 +106,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bars + kBarS + 8 * x, 1);
-      mbar_init(bars + kBarSF + 8 * x, 256);
-      mbar_init(bars + kBarP + 8 * x, 256);
+      mbar_init(bars + kBarSF + 8 * x, 128);
+      mbar_init(bars + kBarP + 8 * x, 128);
       mbar_init(bars + kBarPV + 8 * x, 1);
-      mbar_init(bars + kBarRed + 16 * x, 256);
-      mbar_init(bars + kBarRed + 16 * x + 8, 256);
-      mbar_init(bars + kBarL + 8 * x, 256);
     }
     mbar_init(bars + kBarDrain, 1);
     *abort = 0;
@@ -213,122 +199,103 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       wait_drain(bars + kBarDrain, 0);
     }
   } else {
-    // ---------------- softmax, one query row per thread, half the columns ----------------
-    const int x = warp >> 3, h = (warp >> 2) & 1, wr = warp & 3;
+    // ---------------- softmax, one query row (128 columns) per thread ----------------
+    const int x = warp >> 2, wr = warp & 3;
     const int r = wr * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
-    const uint32_t tS = lane_base + x * kRows + 64 * h, tO = lane_base + kColO + x * kD + 32 * h;
-    const uint32_t tP = lane_base + kColP + x * (kRows / 2) + 32 * h;
+    const uint32_t tS = lane_base + x * kRows, tO = lane_base + kColO + x * kD;
+    const uint32_t tP = lane_base + kColP + x * (kRows / 2);
     const int n = x ? nB : nA;
     const int qrow = q0 + x * kRows + r;
-    float* red = reinterpret_cast<float*>(gbase + kOffRed);
-    float* lsum = reinterpret_cast<float*>(gbase + kOffL);
+    const float2 sc2 = make_float2(sl2, sl2);
     float m_ref = -INFINITY;
-    float2 l2 = make_float2(0.f, 0.f);  // this half's row sum, two partial sums
+    float2 l2 = make_float2(0.f, 0.f);  // row sum, two partial sums
     bool ok = true;
-    bool pv_seen = true;  // the previous P V product is known complete
     for (int j = 0; j < n; ++j) {
       ok = mbar_wait(bars + kBarS + 8 * x, j & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;  // warp-uniform before TMEM access
       tc_fence_after();
-      pv_seen = j == 0;
-      const bool diag = j == n - 1;
-      // Keys after this query (only on the diagonal tile) are masked:
-      // columns c of this half with 64 h + c > lim.
-      const int lim = diag ? qrow - j * kRows - 64 * h : kRows;
-      float v[2][32];
-      tmem_ld32(tS, v[0]);
-      tmem_ld32(tS + 32, v[1]);
-      tmem_wait_ld();
-      if (diag) {
+      float v[4][32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (e > lim) v[0][e] = -INFINITY;
-          if (32 + e > lim) v[1][e] = -INFINITY;
-        }
-      }
-      // Row maximum of the raw scores over this half (sl2 > 0 keeps the
-      // order), then over both halves through shared memory.
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) mx = max3f(mx, fmax3f(v[0][e], v[0][e + 1], v[1][e]), v[1][e + 1]);
-      float* rj = red + ((j & 1) * 4 + x * 2) * kRows;
-      rj[h * kRows + r] = mx;
-      mbar_arrive(bars + kBarRed + 16 * x + 8 * (j & 1));
-      ok = mbar_wait(bars + kBarRed + 16 * x + 8 * (j & 1), (j >> 1) & 1, abort, status);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      mx = fmaxf(mx, rj[(h ^ 1) * kRows + r]) * sl2;
-      const float m_new = mx > m_ref + kRescale ? mx : m_ref;
-      const float alpha = exp2f(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
-      if (j > 0 && __any_sync(0xffffffffu, m_new != m_ref)) {
-        // O_x holds P V up to tile j-1: that product must be complete
-        ok = mbar_wait(bars + kBarPV + 8 * x, (j - 1) & 1, abort, status);
-        if (!(ok = __all_sync(0xffffffffu, ok))) break;
-        pv_seen = true;
-        tc_fence_after();
-        float o[32];
-        tmem_ld32(tO, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-        tmem_st32(tO, o);
-        tmem_wait_st();
-      }
-      m_ref = m_new;
-      l2.x *= alpha;
-      l2.y *= alpha;
-      // P = 2^(s*sl2 - m_ref), row sum, bf16 P.  S is read from TMEM again
-      // rather than kept live across the exchange, then released.
-      tmem_ld32(tS, v[0]);
-      tmem_ld32(tS + 32, v[1]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(bars + kBarSF + 8 * x);
-      if (diag) {
+      mbar_arrive(bars + kBarSF + 8 * x);  // S_x free for the next key tile
+      if (j == n - 1) {  // diagonal tile: keys after this query are masked
+        const int lim = qrow - j * kRows;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (e > lim) v[0][e] = -INFINITY;
-          if (32 + e > lim) v[1][e] = -INFINITY;
-        }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (32 * c + e > lim) v[c][e] = -INFINITY;
       }
-      uint32_t w[32];
-      exp_row(v, sl2, m_ref, l2, w);
-      // P_x(j-1) must have been consumed before it is overwritten
-      if (!pv_seen) {
+      // Row maximum of the raw scores (sl2 > 0 keeps the order).
+      const float mx = row_max(v) * sl2;
+      const float m_new = mx > m_ref + kRescale ? mx : m_ref;
+      const float alpha = exp2f(m_ref - m_new);  // 1 when unchanged, 0 on the first tile
+      // P_x(j-1) V_{j-1} must be complete before P_x is rewritten or O_x rescaled
+      if (j > 0) {
         ok = mbar_wait(bars + kBarPV + 8 * x, (j - 1) & 1, abort, status);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        tc_fence_after();
       }
-      tc_fence_after();
-      tmem_st32u(tP, w);
+      // P = 2^(s*sl2 - m_new): row sum, bf16 P into TMEM 32 columns at a time
+      const float2 nm2 = make_float2(-m_new, -m_new);
+      float2 part[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float2 t = ffma2(make_float2(v[c][e], v[c][e + 1]), sc2, nm2);
+          t.x = ex2_approx(t.x);
+          t.y = ex2_approx(t.y);
+          part[(e >> 1) & 1] = fadd2(part[(e >> 1) & 1], t);
+          w[e >> 1] = pack_bf16x2(t.x, t.y);
+        }
+        tmem_st16(tP + 16 * c, w);
+      }
+      // O_x and the row sum follow a grown reference maximum (O_x is not
+      // touched by an MMA until this tile's P arrives below)
+      if (j > 0 && __any_sync(0xffffffffu, m_new != m_ref)) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      m_ref = m_new;
+      l2 = ffma2(l2, make_float2(alpha, alpha), fadd2(part[0], part[1]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + kBarP + 8 * x);
     }
-    // Row sum over both halves.
-    if (ok) {
-      lsum[(x * 2 + h) * kRows + r] = l2.x + l2.y;
-      mbar_arrive(bars + kBarL + 8 * x);
-      ok = mbar_wait(bars + kBarL + 8 * x, 0, abort, status);
-    }
     if (ok) ok = mbar_wait(bars + kBarPV + 8 * x, (n - 1) & 1, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
-      const float l = lsum[(x * 2) * kRows + r] + lsum[(x * 2 + 1) * kRows + r];
+      const float l = l2.x + l2.y;
       tc_fence_after();
-      float o[32];
-      tmem_ld32(tO, o);
-      tmem_wait_ld();
-      if (qrow < S) {
-        const float inv = 1.f / l;
-        bf16* dst = O + ((int64_t)row0 + qrow) * kD + 32 * h;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t w[4];
+      for (int h = 0; h < 2; ++h) {
+        float o[32];
+        tmem_ld32(tO + 32 * h, o);
+        tmem_wait_ld();
+        if (qrow < S) {
+          const float inv = 1.f / l;
+          bf16* dst = O + ((int64_t)row0 + qrow) * kD + 32 * h;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = pack_bf16x2(o[8 * c + 2 * q] * inv, o[8 * c + 2 * q + 1] * inv);
-          reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) w[q] = pack_bf16x2(o[8 * c + 2 * q] * inv, o[8 * c + 2 * q + 1] * inv);
+            reinterpret_cast<uint4*>(dst)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
-        if (h == 0) lse[(int64_t)row0 + qrow] = (m_ref + log2f(l)) * kLn2;
       }
+      if (qrow < S) lse[(int64_t)row0 + qrow] = (m_ref + log2f(l)) * kLn2;
     }
   }
 
