@@ -431,7 +431,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_extras:
         fwd_ms, _ = timed_steps(layer, stp, args.steps, backward=False)
         extras[w.name] = workload_extras(w, fwd_ms, ms)
-        del layer, Q, K, V, dO, hQ, hK, hV, hdO, hO, hdQ, hdK, hdV, dQ, dK, dV, O
+        del layer, Q, K, V, dO, hQ, hK, hV, hdO, hO, hdQ, hdK, hdV
         torch.cuda.empty_cache()
         if w.name != "512k_k2048":
             w5 = WORKLOADS["512k_k2048"]
