@@ -13,7 +13,7 @@ import torch
 from oracle import lighthouse as oracle
 from long_context_hierarchical_b200.synth import make_inputs, make_scores
 from tests.helpers import (TOL, assert_close, assert_grad_close, assert_pyr_close,
-                           grad_tolerance_terms, np64, oracle_layer, stack)
+                           grad_term_bounds, grad_tolerance_terms, np64, oracle_layer, stack)
 
 pytestmark = pytest.mark.gpu
 
@@ -254,6 +254,37 @@ def test_whole_layer(case):
         assert_grad_close(np64(got), c["grads"][i], c["terms"][key], dt, key)
     for a, b in zip(g3, g4):
         assert torch.equal(a, b)
+    lh.device_status()
+
+
+@pytest.mark.parametrize("S", [1000, 2304])
+def test_attention_with_growing_row_maxima(S):
+    """Keys whose scale grows along the sequence make each query's running
+    maximum rise by many powers of two across key tiles, so the forward's
+    lazy rescaling of O (only when the maximum grows by more than 2^8) runs
+    repeatedly; forward and backward against the oracle in fp64."""
+    from long_context_hierarchical_b200 import lh
+    BH = 2
+    g = np.random.default_rng(7)
+    ramp = (1.0 + 5.0 * np.arange(S) / S)[None, :, None]
+    Q = oracle.round_bf16(g.standard_normal((BH, S, 64)))
+    K = oracle.round_bf16(g.standard_normal((BH, S, 64)) * ramp)
+    V = oracle.round_bf16(g.standard_normal((BH, S, 64)))
+    dO = oracle.round_bf16(g.standard_normal((BH, S, 64)))
+    dev = [_t(x, torch.bfloat16) for x in (Q, K, V, dO)]
+    O, lse = lh.attn_fwd(*dev[:3])
+    grads = lh.attn_bwd(*dev[:3], O, lse, dev[3], None)
+    torch.cuda.synchronize()
+    for b in range(BH):
+        Oe, lse_e = oracle.causal_attention(Q[b], K[b], V[b])
+        Ob = oracle.round_bf16(Oe)
+        D = np.sum(dO[b] * Ob, axis=1)
+        ge = oracle.causal_attention_bwd(Q[b], K[b], V[b], dO[b], lse_e, D)
+        mq, mk, mv, mo = grad_term_bounds(Q[b], K[b], V[b], Ob, lse_e, dO[b])
+        assert np.max(np.abs(np64(lse[b]) - lse_e)) <= 1e-3
+        assert_grad_close(np64(O[b]), Oe, mo, torch.bfloat16, f"O (head {b})")
+        for got, exp, m, name in zip(grads, ge, (mq, mk, mv), ("dQ", "dK", "dV")):
+            assert_grad_close(np64(got[b]), exp, m, torch.bfloat16, f"{name} (head {b})")
     lh.device_status()
 
 
