@@ -136,12 +136,16 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
   for (int k = 0; k < kChunks; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
 }
 
+constexpr int kBwdLanes = 4;  // lanes per slot row in the scatter backward (8 and 2 measured slower)
+constexpr int kBwdChunks = 8 / kBwdLanes;
+constexpr int kRowsPerBlockB = kThreads / kBwdLanes;
+
 template <typename T, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
                    const int32_t* __restrict__ sel_idx, T* __restrict__ dOg, float* __restrict__ D) {
-  const int j = blockIdx.x * kRowsPerBlock + (threadIdx.x >> 3);
-  const int c = threadIdx.x & 7;
+  const int j = blockIdx.x * kRowsPerBlockB + (int)(threadIdx.x / kBwdLanes);
+  const int c = threadIdx.x % kBwdLanes;
   const int S = (int)g.S, N = (int)g.N;
   const bool live = j < S;
   const int64_t bh = blockIdx.y;
@@ -157,35 +161,47 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   const int lo = ((i + 1) << sh) - 1;
   const int hi = min(lo + (1 << sh) - 1, N - 1);
   const T* src = dO + bh * g.N * kD + c * 8;
-  float acc[8];
+  float acc[kBwdChunks][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int k = 0; k < kBwdChunks; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
   int t = lo;
   for (; t + 3 <= hi; t += 4) {  // four independent row loads in flight
-    float x0[8], x1[8], x2[8], x3[8];
-    Vec8<T>::load(src + (int64_t)t * kD, x0);
-    Vec8<T>::load(src + (int64_t)(t + 1) * kD, x1);
-    Vec8<T>::load(src + (int64_t)(t + 2) * kD, x2);
-    Vec8<T>::load(src + (int64_t)(t + 3) * kD, x3);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += ((x0[e] + x1[e]) + (x2[e] + x3[e]));
+    for (int k = 0; k < kBwdChunks; ++k) {
+      float x0[8], x1[8], x2[8], x3[8];
+      const T* p = src + 8 * kBwdLanes * k;
+      Vec8<T>::load(p + (int64_t)t * kD, x0);
+      Vec8<T>::load(p + (int64_t)(t + 1) * kD, x1);
+      Vec8<T>::load(p + (int64_t)(t + 2) * kD, x2);
+      Vec8<T>::load(p + (int64_t)(t + 3) * kD, x3);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] += ((x0[e] + x1[e]) + (x2[e] + x3[e]));
+    }
   }
   for (; t <= hi; ++t) {
-    float x[8];
-    Vec8<T>::load(src + (int64_t)t * kD, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += x[e];
+    for (int k = 0; k < kBwdChunks; ++k) {
+      float x[8];
+      Vec8<T>::load(src + 8 * kBwdLanes * k + (int64_t)t * kD, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[k][e] += x[e];
+    }
   }
-  float o[8];
-  Vec8<T>::load(Og + r * kD + c * 8, o);
   float dsum = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) dsum = fmaf(Vec8<T>::rounded(acc[e]), o[e], dsum);
-  dsum += __shfl_xor_sync(0xffffffffu, dsum, 1);
-  dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
-  dsum += __shfl_xor_sync(0xffffffffu, dsum, 4);
+  for (int k = 0; k < kBwdChunks; ++k) {
+    float o[8];
+    Vec8<T>::load(Og + r * kD + c * 8 + 8 * kBwdLanes * k, o);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dsum = fmaf(Vec8<T>::rounded(acc[k][e]), o[e], dsum);
+  }
+#pragma unroll
+  for (int m = 1; m < kBwdLanes; m <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
   if (!live) return;
-  Vec8<T>::store(dOg + r * kD + c * 8, acc);
+#pragma unroll
+  for (int k = 0; k < kBwdChunks; ++k) Vec8<T>::store(dOg + r * kD + c * 8 + 8 * kBwdLanes * k, acc[k]);
   if (c == 0) D[r] = dsum;
 }
 
@@ -298,7 +314,7 @@ cudaError_t launch_scatter(const lh_plan& plan, const void* Og, const int32_t* s
 template <typename T>
 void scatter_bwd_t(const Geo& g, const void* dO, const void* Og, const int32_t* sel_idx, void* dOg,
                    float* D, cudaStream_t st) {
-  const dim3 grid((unsigned)((g.S + kRowsPerBlock - 1) / kRowsPerBlock), (unsigned)g.BH);
+  const dim3 grid((unsigned)((g.S + kRowsPerBlockB - 1) / kRowsPerBlockB), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
     scatter_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og, sel_idx,
                                                               (T*)dOg, D);
