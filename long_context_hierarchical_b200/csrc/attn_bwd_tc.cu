@@ -7,31 +7,32 @@
 //   dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d).
 // Two schedules:
 //  - fused (default): one kernel.  A CTA per 128-key tile streams query
-//    chunks of C rows from its diagonal on.  S^T = K Q^T and dP^T = V dO^T
-//    land in TMEM (lane = key); the element-wise warps turn them into P^T
-//    and dS^T (bf16, swizzled K-major smem); dV += P^T dO and dK += dS^T Q
-//    accumulate in TMEM, and the chunk's dQ share dS K (the dS^T tile read
-//    MN-major as the A operand) lands in TMEM, from where the element-wise
-//    warps add it into an fp32 dQ accumulator in global memory (fp32
-//    atomics, so the summation order, and the last bits of dQ, vary from
-//    run to run).  A small kernel scales and rounds the accumulator to dQ.
-//    P and dS are formed once per (key, query) pair.
+//    chunks of 128 rows from its diagonal on.  S^T = K Q^T and dP^T = V dO^T
+//    land in TMEM (lane = key), with lse and D folded in by one extra MMA
+//    step (see the K=16 slices below); the element-wise warps turn them into
+//    P^T (bf16, TMEM: the A operand of dV += P^T dO) and dS^T (bf16, swizzled
+//    K-major smem: the A operand of dK += dS^T Q and, read MN-major, of the
+//    chunk's dQ share dS K, which lands in TMEM).  dV and dK accumulate in
+//    TMEM; each dQ share is staged through shared memory and reduce-added by
+//    TMA into an fp32 dQ accumulator in global memory, whose summation order
+//    (and so the last bits of dQ) varies from run to run.  A small kernel
+//    scales and rounds the accumulator into dQ.  P and dS are formed once
+//    per (key, query) pair: exactly the five products of the gradient.
 //  - deterministic: two kernels, no atomics.  The dk/dv kernel above without
 //    the dQ share, then a dq kernel: one CTA per 128-query tile streams key
-//    chunks of C rows up to its diagonal; S = Q K^T and dP = dO V^T in TMEM
-//    (lane = query), dS to smem, dQ += dS K in TMEM.  P and dS are formed
-//    twice.
-// Warp roles: C/32 element-wise groups of four warps split each step's C
+//    chunks up to its diagonal; S = Q K^T and dP = dO V^T in TMEM (lane =
+//    query), dS to smem, dQ += dS K in TMEM.  P and dS are formed twice.
+// Warp roles: four element-wise groups of four warps split each step's 128
 // columns (no row reductions are needed here), then one load warp (TMA for
-// tiles, plain loads for LSE/D) and one warp that owns TMEM and issues the
-// MMAs from one thread.  With C = 64 the TMEM (<= 256 columns) and shared
-// memory of a CTA fit twice on an SM, so two independent CTAs interleave
-// their MMA / element-wise / load latencies.
+// tiles; it also writes the per-chunk lse and D slices) and one warp that
+// owns TMEM and issues the MMAs (and, fused, the dQ reduce-adds) from one
+// thread.
 // Overlap inside a CTA: each element-wise thread copies its S/dP columns out
 // of TMEM and releases them at once, so the next step's S and dP MMAs run
-// while it computes; the single P/dS shared-memory tile has its own
-// "consumed" barrier that the element-wise warps wait on just before
-// overwriting it.
+// while it computes; the P^T / dS^T buffers have their own "consumed"
+// barrier that the element-wise warps wait on just before overwriting them,
+// and the dQ share of one step is staged while the next step's dV/dK MMAs
+// run.
 // Operand layouts are those of the forward kernel: K-major A/B tiles with the
 // 128-byte swizzle, tiles read as the MN-major B operand (dO, Q, K) with
 // 8-row groups 1024 bytes apart.  Every wait is bounded (see tc.cuh).
