@@ -44,6 +44,8 @@ WORKLOADS = {
     "98k_k1536": Workload("98k_k1536", 1, 16, 98304, 64, "bf16", 4, 3, 1536, True),
     "98k_k6144": Workload("98k_k6144", 1, 16, 98304, 64, "bf16", 4, 3, 6144, True),
     "512k_k2048": Workload("512k_k2048", 1, 16, 524288, 64, "bf16", 4, 4, 2048, True),
+    # the pages' best pyramid ablation (pooling factor 2) at the 98K length: S = 30720
+    "98k_p2_k1536": Workload("98k_p2_k1536", 1, 16, 98304, 64, "bf16", 2, 3, 1536, True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}

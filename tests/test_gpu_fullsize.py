@@ -48,7 +48,7 @@ def _check(got, exp, terms, what):
                            f"max abs err {err.max():.3e}")
 
 
-@pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048"])
+@pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048", "98k_p2_k1536"])
 def run(request):
     from long_context_hierarchical_b200 import lh
     w = WORKLOADS[request.param]
