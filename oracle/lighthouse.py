@@ -31,6 +31,12 @@ Readings of points the pages leave open (each marked READING below):
   R5 uncovered output positions are 0; R(l, i) is clipped to N-1.
   R6 selection is per (batch, head).
   R7 scatter sums levels in ascending order, without atomics.
+  R8 (alternative selection, rule "descent") hierarchical descent: keep
+     every coarsest entry; at the coarsest level pick the k best entries,
+     keep their p children one level down, pick the k best of those, and so
+     on to level 0.  Another reading of the budget (L-1)*p*k: p*k entries per
+     finer level.  Needs k <= N/p^(L-1).  Coarse scores are the same
+     max-pools as in R1; ties as in R3.
 """
 from __future__ import annotations
 
@@ -192,6 +198,36 @@ def select(cand, sz: Sizes):
     mask = np.zeros(sz.Ntot, dtype=bool)
     mask[order[: sz.Ksel]] = True
     mask[sz.flat_off[sz.L - 1]:] = True
+    return mask
+
+
+def select_descent(cand, sz: Sizes):
+    """Boolean mask over all Ntot entries for the hierarchical descent (READING R8).
+
+    ``cand`` holds the scores of levels 0..L-2 (level-major, as from
+    ``candidate_scores``); a level-(L-1) entry's score is the maximum of its p
+    children's, i.e. of its span's level-0 scores, the same max-pool.  From
+    the coarsest level down: the k best of the current entries (ties to the
+    lower flat index) pass their p children to the next level down, which
+    are all kept; at level 0 the descent stops.
+    """
+    L, p, k = sz.L, sz.p, sz.k
+    mask = np.zeros(sz.Ntot, dtype=bool)
+    mask[sz.flat_off[L - 1]:] = True
+    if L < 2 or k == 0:
+        return mask
+    if k > sz.n[L - 1]:
+        raise ValueError("descent needs k <= N/p^(L-1)")
+    cand = np.asarray(cand, dtype=np.float64)
+    top = cand[sz.flat_off[L - 2]: sz.flat_off[L - 1]].reshape(sz.n[L - 1], p).max(axis=1)
+    current = np.arange(sz.n[L - 1], dtype=np.int64)  # entries of level l, ascending
+    cur_scores = top
+    for l in range(L - 1, 0, -1):
+        best = current[np.argsort(-cur_scores, kind="stable")[:k]]
+        children = np.sort((best[:, None] * p + np.arange(p)[None, :]).ravel())
+        mask[sz.flat_off[l - 1] + children] = True
+        current = children
+        cur_scores = cand[sz.flat_off[l - 1] + children]
     return mask
 
 
@@ -368,23 +404,25 @@ def gather_bwd(dXg, slot_of, sz: Sizes, mode: str):
 # ---------------------------------------------------------------------------
 
 
-def head_select(Qh, Kh, sz: Sizes):
-    """Scores, mask and order of one head (stages 2 and the ordering of 3)."""
+def head_select(Qh, Kh, sz: Sizes, rule: str = "joint"):
+    """Scores, mask and order of one head (stages 2 and the ordering of 3).
+
+    rule: "joint" (READING R2) or "descent" (READING R8)."""
     s0 = level0_scores(Qh, Kh)
     cand = candidate_scores(s0, sz)
-    mask = select(cand, sz)
+    mask = select(cand, sz) if rule == "joint" else select_descent(cand, sz)
     sel_idx, slot_of = order_selection(mask, sz)
     return cand, sel_idx, slot_of
 
 
-def head_forward(Qh, Kh, Vh, sz: Sizes, mode: str, selection=None):
+def head_forward(Qh, Kh, Vh, sz: Sizes, mode: str, selection=None, rule: str = "joint"):
     """One head's forward.  ``selection`` = (sel_idx, slot_of) freezes stage 2."""
     Qh = np.asarray(Qh, dtype=np.float64)
     Kh = np.asarray(Kh, dtype=np.float64)
     Vh = np.asarray(Vh, dtype=np.float64)
     pq, pk, pv = pyramid(Qh, sz, mode), pyramid(Kh, sz, mode), pyramid(Vh, sz, mode)
     if selection is None:
-        cand, sel_idx, slot_of = head_select(Qh, Kh, sz)
+        cand, sel_idx, slot_of = head_select(Qh, Kh, sz, rule)
     else:
         cand = None
         sel_idx, slot_of = selection
@@ -408,12 +446,12 @@ def head_backward(ctx, dOh, sz: Sizes, mode: str):
     return dict(dOg=dOg, D=D, dQg=dQg, dKg=dKg, dVg=dVg, dQ=dQ, dK=dK, dV=dV)
 
 
-def forward(Q, K, V, p: int, L: int, k: int, mode: str):
+def forward(Q, K, V, p: int, L: int, k: int, mode: str, rule: str = "joint"):
     """Whole layer forward over [B, H, N, d] arrays; returns per-head contexts."""
     Q = np.asarray(Q, dtype=np.float64)
     B, H, N, d = Q.shape
     sz = sizes(N, p, L, k)
-    ctxs = [[head_forward(Q[b, h], K[b, h], V[b, h], sz, mode) for h in range(H)]
+    ctxs = [[head_forward(Q[b, h], K[b, h], V[b, h], sz, mode, rule=rule) for h in range(H)]
             for b in range(B)]
     O = np.stack([np.stack([c["O"] for c in row]) for row in ctxs])
     return O, ctxs, sz

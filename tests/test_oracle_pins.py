@@ -246,6 +246,68 @@ def test_selection_invariants_random():
         assert cand[parent] >= thr
 
 
+def test_descent_hand_worked():
+    """Hierarchical descent (reading R8) on a hand-worked case, which the joint
+    rule selects differently."""
+    g = GOLDEN["descent"]
+    sz = lh.sizes(g["N"], g["p"], g["L"], g["k"])
+    cand = lh.candidate_scores(np.array(g["s0"], float), sz)
+    sel_idx, _ = lh.order_selection(lh.select_descent(cand, sz), sz)
+    assert sel_idx.tolist() == g["sel_idx"]
+    joint, _ = lh.order_selection(lh.select(cand, sz), sz)
+    assert joint.tolist() == g["joint_sel_idx"]
+    t = GOLDEN["descent_ties"]
+    sz = lh.sizes(t["N"], t["p"], t["L"], t["k"])
+    cand = lh.candidate_scores(np.array(t["s0"], float), sz)
+    sel_idx, _ = lh.order_selection(lh.select_descent(cand, sz), sz)
+    assert sel_idx.tolist() == t["sel_idx"]
+
+
+@pytest.mark.parametrize("p", [2, 4])
+def test_descent_two_levels_is_best_blocks(p):
+    """L = 2: the level-0 tokens kept are exactly the spans of the k blocks
+    with the largest maximum token score (ties to the lower block)."""
+    N, k = 64 * p, 5
+    sz = lh.sizes(N, p, 2, k)
+    s0 = rng(3).integers(0, 6, N).astype(float)
+    mask = lh.select_descent(lh.candidate_scores(s0, sz), sz)
+    blocks = sorted(range(N // p), key=lambda b: (-max(s0[b * p:(b + 1) * p]), b))[:k]
+    exp = {b * p + c for b in blocks for c in range(p)} | set(range(sz.flat_off[1], sz.Ntot))
+    assert set(np.nonzero(mask)[0].tolist()) == exp
+
+
+@pytest.mark.parametrize("p,L,k,distinct", [(2, 4, 3, None), (4, 3, 4, 3), (2, 5, 2, 2), (4, 4, 2, None)])
+def test_descent_invariants_random(p, L, k, distinct):
+    """Per finer level exactly p*k entries; each is a child of an entry one
+    level up that is kept; those parents are the k best of their level's
+    kept entries under (score desc, index asc)."""
+    N = 64 * p ** (L - 1)
+    sz = lh.sizes(N, p, L, k)
+    r = rng(11)
+    s0 = r.random(N) if distinct is None else r.integers(0, distinct, N).astype(float)
+    cand = lh.candidate_scores(s0, sz)
+    mask = lh.select_descent(cand, sz)
+    assert mask.sum() == sz.S
+    assert mask[sz.flat_off[L - 1]:].all()
+    # scores of every level, by max-pooling level 0 directly
+    score = [s0.reshape(sz.n[l], sz.P[l]).max(axis=1) for l in range(L)]
+    for l in range(L - 1):
+        kept = np.nonzero(mask[sz.flat_off[l]:sz.flat_off[l + 1]])[0]
+        assert kept.size == p * k
+        parents = np.unique(kept // p)
+        assert parents.size == k and np.array_equal(np.sort(kept), np.sort((parents[:, None] * p + np.arange(p)).ravel()))
+        up = np.nonzero(mask[sz.flat_off[l + 1]:sz.flat_off[l + 2]])[0]  # kept entries one level up
+        assert set(parents.tolist()) <= set(up.tolist())
+        ranked = sorted(up.tolist(), key=lambda i: (-score[l + 1][i], i))
+        assert set(ranked[:k]) == set(parents.tolist())
+
+
+def test_descent_needs_k_within_the_coarsest_level():
+    sz = lh.sizes(64, 2, 4, 9)  # n_3 = 8 < k
+    with pytest.raises(ValueError):
+        lh.select_descent(np.zeros(sz.M), sz)
+
+
 # --------------------------------------------------------------------------
 # stage 3: attention
 # --------------------------------------------------------------------------
