@@ -114,7 +114,7 @@ class Layer:
     def __init__(self, lh, w, Q, K, V, dO):
         import ctypes
         self.lh, self.w = lh, w
-        self.pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+        self.pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype, select=w.select)
         self.Q, self.K, self.V, self.dO = Q, K, V, dO
         dev = Q.device
         self.ctx = lh.Context(self.pl, dev)
@@ -194,7 +194,7 @@ def oracle_head_seconds(w, Qh, Kh, Vh, dOh):
     mode = "bf16" if w.dtype == "bf16" else "f32"
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     t0 = time.perf_counter()
-    ctx = oracle.head_forward(Qh, Kh, Vh, sz, mode)
+    ctx = oracle.head_forward(Qh, Kh, Vh, sz, mode, rule=w.select)
     oracle.head_backward(ctx, dOh, sz, mode)
     return time.perf_counter() - t0
 

@@ -74,9 +74,20 @@ typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
  * (level 0 = tokens), k: per-level budget unit, so (L-1)*p*k entries are
  * selected (skill card, "阶段 3").  The method needs N to be a multiple of
  * p^(L-1).  Built here: d = 64, p in {2, 4}, 1 <= L <= 5, p^(L-1) <= 256. */
+/* Selection rule for the (L-1)*p*k budget (lh_config.select):
+ *  LH_SELECT_JOINT   one top-K of (L-1)*p*k over all candidate levels
+ *                    0..L-2 (the default reading);
+ *  LH_SELECT_DESCENT hierarchical descent: from the coarsest level down, the
+ *                    k best entries of a level keep their p children one
+ *                    level down (p*k per finer level); needs k <= n[L-1].
+ * Both keep every coarsest-level entry and break ties to the lower
+ * level-major flat index (skill card "阶段 2", "阶段 3"). */
+typedef enum { LH_SELECT_JOINT = 0, LH_SELECT_DESCENT = 1 } lh_select;
+
 typedef struct {
   int32_t B, H, N, d, p, L, k;
-  int32_t dtype; /* lh_dtype */
+  int32_t dtype;  /* lh_dtype */
+  int32_t select; /* lh_select */
 } lh_config;
 
 /* Sizes and buffer layout derived from a config by lh_plan_init.
@@ -107,8 +118,9 @@ typedef struct {
 
 /* Fill *out from *cfg.  Host only, enqueues nothing.  Returns
  * LH_ERR_INVALID_ARG when the method itself is undefined for the config
- * (N % p^(L-1) != 0, L < 1, p < 2, k < 0, (L-1)*p*k > M, S >= 2^31) and
- * LH_ERR_UNSUPPORTED for shapes this build does not implement. */
+ * (N % p^(L-1) != 0, L < 1, p < 2, k < 0, (L-1)*p*k > M, S >= 2^31, an
+ * unknown select, descent with k > n[L-1]) and LH_ERR_UNSUPPORTED for
+ * shapes this build does not implement. */
 lh_status lh_plan_init(const lh_config* cfg, lh_plan* out);
 
 /* Stage 1 (skill card "阶段 1"; gist.science 2.A).  Writes pyramid levels

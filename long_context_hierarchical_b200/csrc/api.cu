@@ -50,6 +50,8 @@ Geo make_geo(const lh_plan& p) {
   g.L = p.c.L;
   g.p = p.c.p;
   g.logp = p.c.p == 2 ? 1 : 2;
+  g.k = p.c.k;
+  g.select = p.c.select;
   for (int l = 0; l < LH_MAX_LEVELS; ++l) {
     g.n[l] = p.n[l];
     g.pyr_off[l] = p.pyr_off[l];
@@ -128,6 +130,10 @@ lh_status lh_plan_init(const lh_config* cfg, lh_plan* out) {
   p.Ksel = (int64_t)(c.L - 1) * c.p * c.k;
   if (p.Ksel > p.M) return fail(LH_ERR_INVALID_ARG, "(L-1)*p*k exceeds the candidate count");
   p.S = p.n[c.L - 1] + p.Ksel;
+  if (c.select != LH_SELECT_JOINT && c.select != LH_SELECT_DESCENT)
+    return fail(LH_ERR_INVALID_ARG, "select must be LH_SELECT_JOINT or LH_SELECT_DESCENT");
+  if (c.select == LH_SELECT_DESCENT && c.L >= 2 && c.k > p.n[c.L - 1])
+    return fail(LH_ERR_INVALID_ARG, "descent selection needs k <= N / p^(L-1)");
   if (p.S >= (int64_t(1) << 31) || p.Ntot >= (int64_t(1) << 31))
     return fail(LH_ERR_INVALID_ARG, "S and the pyramid size must stay below 2^31");
   p.elem_bytes = c.dtype == LH_BF16 ? 2 : 4;

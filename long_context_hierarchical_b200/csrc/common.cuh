@@ -79,6 +79,7 @@ struct Vec8<float> {
 struct Geo {
   int64_t BH, N, S, Ntot, Npyr, M, Ksel;
   int L, p, logp;
+  int k, select;  // per-level budget and lh_select rule
   int64_t n[LH_MAX_LEVELS];
   int64_t flat_off[LH_MAX_LEVELS + 1];
   int64_t pyr_off[LH_MAX_LEVELS];

@@ -22,9 +22,20 @@
 // ((t + 1) % p^l == 0).  A count per token block, a scan of the block counts
 // and a rewrite give each selected entry its slot with no sort.
 //
+// Hierarchical descent (lh_select LH_SELECT_DESCENT, the other reading of
+// the (L-1)*p*k budget): one block per (batch, head) walks from the coarsest
+// level down; at each level it finds the k-th largest key among the level's
+// kept entries by an exact 8-bit radix select over the 64-bit keys, keeps
+// the p children of the entries at or above it (a byte mask over the
+// candidates) and continues with those children.  A coarsest entry's score
+// is the maximum of its p children's, the same max-pool as the candidates'.
+// The ordering kernels then read the mask instead of a threshold.
+//
 // Grid-wide phases are separate launches, and the reduction that closes a
 // phase runs in the last block to finish (an atomic ticket); no block ever
 // waits for another.
+#include <algorithm>
+
 #include "host.h"
 
 namespace lh {
@@ -48,8 +59,11 @@ struct HeadState {
 };
 static_assert(sizeof(HeadState) == 64, "HeadState is 64 bytes");
 
+constexpr int kDescThreads = 1024;
+
 struct Layout {
-  int64_t hist1, hist2, state, blockcnt, list, zero_bytes, total;
+  int64_t hist1, hist2, state, blockcnt, list, mask, keys, zero_bytes, total;
+  int64_t cap;  // descent: keys per level list
 };
 
 int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
@@ -66,6 +80,13 @@ Layout layout(const lh_plan& p) {
   o = align256(o);
   l.blockcnt = o; o = align256(o + BH * nblk * 4);
   l.list = o; o = align256(o + BH * p.M * 8);
+  l.cap = 0;
+  l.mask = l.keys = o;
+  if (p.c.select == LH_SELECT_DESCENT && p.c.L >= 2) {
+    l.cap = std::max<int64_t>(p.n[p.c.L - 1], (int64_t)p.c.p * p.c.k);
+    l.mask = o; o = align256(o + BH * p.M);
+    l.keys = o; o = align256(o + BH * 2 * l.cap * 8);
+  }
   l.total = o;
   return l;
 }
@@ -254,18 +275,104 @@ collect_kernel(Geo g, const float* __restrict__ scores, unsigned long long* list
   if (threadIdx.x == 0) st->kappa = ((unsigned long long)prefix << 40) | rem;
 }
 
+// --- hierarchical descent ----------------------------------------------------
+
+// The k-th largest of n unique keys (1 <= k <= n), by eight 8-bit radix passes
+// over the keys from the most significant digit.  Whole block.
+__device__ unsigned long long block_kth_largest(const unsigned long long* keys, int64_t n, uint32_t k,
+                                                uint32_t* h, uint32_t* warp_sums, uint32_t* s_digit,
+                                                uint32_t* s_need) {
+  unsigned long long prefix = 0, pmask = 0;
+  uint32_t need = k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += kDescThreads) h[i] = 0;
+    __syncthreads();
+    for (int64_t j = threadIdx.x; j < n; j += kDescThreads) {
+      const unsigned long long key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&h[(key >> shift) & 0xffu], 1u);
+    }
+    __syncthreads();
+    const int t = threadIdx.x;
+    const uint32_t v = t < 256 ? h[255 - t] : 0;  // descending digits
+    const uint32_t above = block_excl_scan<kDescThreads>(v, warp_sums, nullptr);
+    if (t < 256 && above < need && need <= above + v) {
+      *s_digit = 255 - t;
+      *s_need = need - above;
+    }
+    __syncthreads();
+    prefix |= (unsigned long long)*s_digit << shift;
+    pmask |= 0xffull << shift;
+    need = *s_need;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kDescThreads)
+descent_kernel(Geo g, const float* __restrict__ scores, uint8_t* __restrict__ mask,
+               unsigned long long* __restrict__ keys, int64_t cap) {
+  __shared__ uint32_t h[256];
+  __shared__ uint32_t warp_sums[kDescThreads / 32];
+  __shared__ uint32_t s_digit, s_need;
+  const int64_t bh = blockIdx.x;
+  const float* s = scores + bh * g.M;
+  uint8_t* msk = mask + bh * g.M;
+  unsigned long long* cur = keys + bh * 2 * cap;
+  unsigned long long* nxt = cur + cap;
+  const int L = g.L, p = g.p;
+  const uint32_t k = (uint32_t)g.k;
+  // the coarsest level: score = max over the p children (level L-2)
+  int64_t n = g.n[L - 1];
+  for (int64_t i = threadIdx.x; i < n; i += kDescThreads) {
+    const float* c = s + g.flat_off[L - 2] + i * p;
+    float m = c[0];
+    for (int j = 1; j < p; ++j) m = fmaxf(m, c[j]);
+    cur[i] = full_key(m, g.flat_off[L - 1] + i);
+  }
+  __syncthreads();
+  for (int l = L - 1; l >= 1; --l) {
+    const unsigned long long kappa = block_kth_largest(cur, n, k, h, warp_sums, &s_digit, &s_need);
+    // keep the p children of every entry at or above kappa (exactly k of them)
+    uint32_t base = 0;
+    for (int64_t j0 = 0; j0 < n; j0 += kDescThreads) {
+      const int64_t j = j0 + threadIdx.x;
+      const unsigned long long key = j < n ? cur[j] : 0ull;
+      const bool keep = j < n && key >= kappa;
+      uint32_t total;
+      const uint32_t pos = base + block_excl_scan<kDescThreads>(keep ? 1u : 0u, warp_sums, &total);
+      if (keep) {
+        const int64_t f = 0xffffffffll - (int64_t)(key & 0xffffffffull);  // flat index at level l
+        const int64_t i = f - g.flat_off[l];
+        for (int c = 0; c < p; ++c) {
+          const int64_t child = g.flat_off[l - 1] + i * p + c;
+          msk[child] = 1;
+          if (l - 1 >= 1 && pos < k) nxt[(int64_t)pos * p + c] = full_key(s[child], child);
+        }
+      }
+      base += total;
+    }
+    __syncthreads();
+    unsigned long long* t = cur;
+    cur = nxt;
+    nxt = t;
+    n = (int64_t)p * k;
+  }
+}
+
 // --- ordering -------------------------------------------------------------
 
 struct SelCtx {
-  const float* s;  // this head's candidate scores
+  const float* s;      // this head's candidate scores
+  const uint8_t* msk;  // descent: this head's candidate mask (else null)
   unsigned long long kappa;
-  bool any;        // Ksel > 0
+  bool any;            // Ksel > 0
 };
 
 __device__ __forceinline__ bool is_selected(const Geo& g, const SelCtx& c, int l, int64_t i) {
   if (l == g.L - 1) return true;
   if (!c.any) return false;
   const int64_t f = g.flat_off[l] + i;
+  if (c.msk) return c.msk[f] != 0;
   return full_key(c.s[f], f) >= c.kappa;
 }
 
@@ -283,11 +390,11 @@ __device__ __forceinline__ uint32_t count_range(const Geo& g, const SelCtx& c, i
 }
 
 __global__ void __launch_bounds__(kOrdThreads)
-order_count_kernel(Geo g, const float* __restrict__ scores, const HeadState* state,
-                   uint32_t* blockcnt, HeadState* wstate, int64_t nblk) {
+order_count_kernel(Geo g, const float* __restrict__ scores, const uint8_t* __restrict__ mask,
+                   const HeadState* state, uint32_t* blockcnt, HeadState* wstate, int64_t nblk) {
   __shared__ uint32_t warp_sums[kOrdThreads / 32];
   const int64_t bh = blockIdx.y;
-  SelCtx c{scores + bh * g.M, state[bh].kappa, g.Ksel > 0};
+  SelCtx c{scores + bh * g.M, mask ? mask + bh * g.M : nullptr, state[bh].kappa, g.Ksel > 0};
   const int64_t t0 = (int64_t)blockIdx.x * kTokBlock + threadIdx.x * kTokPerThread;
   const int64_t t1 = min(g.N, t0 + kTokPerThread);
   const uint32_t mine = t0 < g.N ? count_range(g, c, t0, t1) : 0;
@@ -309,12 +416,12 @@ order_count_kernel(Geo g, const float* __restrict__ scores, const HeadState* sta
 }
 
 __global__ void __launch_bounds__(kOrdThreads)
-order_write_kernel(Geo g, const float* __restrict__ scores, const HeadState* state,
-                   const uint32_t* blockoff, int32_t* __restrict__ sel_idx,
+order_write_kernel(Geo g, const float* __restrict__ scores, const uint8_t* __restrict__ mask,
+                   const HeadState* state, const uint32_t* blockoff, int32_t* __restrict__ sel_idx,
                    int32_t* __restrict__ slot_of, int64_t nblk) {
   __shared__ uint32_t warp_sums[kOrdThreads / 32];
   const int64_t bh = blockIdx.y;
-  SelCtx c{scores + bh * g.M, state[bh].kappa, g.Ksel > 0};
+  SelCtx c{scores + bh * g.M, mask ? mask + bh * g.M : nullptr, state[bh].kappa, g.Ksel > 0};
   const int64_t t0 = (int64_t)blockIdx.x * kTokBlock + threadIdx.x * kTokPerThread;
   const int64_t t1 = min(g.N, t0 + kTokPerThread);
   const uint32_t mine = t0 < g.N ? count_range(g, c, t0, t1) : 0;
@@ -359,15 +466,22 @@ cudaError_t launch_topk(const lh_plan& plan, const float* scores, int32_t* sel_i
 
   cudaError_t e = cudaMemsetAsync(w, 0, lay.zero_bytes, st);
   if (e != cudaSuccess) return e;
-  if (g.Ksel > 0) {
+  const bool descent = g.select == LH_SELECT_DESCENT && g.Ksel > 0;
+  uint8_t* mask = descent ? reinterpret_cast<uint8_t*>(w + lay.mask) : nullptr;
+  if (descent) {
+    e = cudaMemsetAsync(mask, 0, (size_t)(g.BH * g.M), st);
+    if (e != cudaSuccess) return e;
+    descent_kernel<<<(unsigned)g.BH, kDescThreads, 0, st>>>(
+        g, scores, mask, reinterpret_cast<unsigned long long*>(w + lay.keys), lay.cap);
+  } else if (g.Ksel > 0) {
     const dim3 grid((unsigned)((g.M + kChunk - 1) / kChunk), (unsigned)g.BH);
     hist1_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, hist1, state);
     hist2_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, hist2, state);
     collect_kernel<<<grid, kSelThreads, 0, st>>>(g, scores, list, state);
   }
   const dim3 ogrid((unsigned)nblk, (unsigned)g.BH);
-  order_count_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, state, blockcnt, state, nblk);
-  order_write_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, state, blockcnt, sel_idx, slot_of,
+  order_count_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, mask, state, blockcnt, state, nblk);
+  order_write_kernel<<<ogrid, kOrdThreads, 0, st>>>(g, scores, mask, state, blockcnt, sel_idx, slot_of,
                                                     nblk);
   return cudaGetLastError();
 }

@@ -32,8 +32,11 @@ EXPORTS = (
 )
 
 
+SELECT = {"joint": 0, "descent": 1}
+
+
 class LhConfig(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "p", "L", "k", "dtype")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "N", "d", "p", "L", "k", "dtype", "select")]
 
 
 _I64 = ctypes.c_int64
@@ -161,8 +164,10 @@ class Plan:
 
 
 def plan(B: int, H: int, N: int, d: int = 64, p: int = 4, L: int = 3, k: int = 0,
-         dtype: str = "bf16") -> Plan:
-    cfg = LhConfig(B, H, N, d, p, L, k, DTYPES[dtype])
+         dtype: str = "bf16", select: str = "joint") -> Plan:
+    """select: "joint" (one top-K over all candidate levels) or "descent"
+    (hierarchical descent from the coarsest level)."""
+    cfg = LhConfig(B, H, N, d, p, L, k, DTYPES[dtype], SELECT[select])
     raw = LhPlan()
     _check(LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(raw)), "lh_plan_init")
     return Plan(raw)

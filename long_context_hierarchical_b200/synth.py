@@ -35,6 +35,7 @@ class Workload:
     L: int
     k: int
     backward: bool
+    select: str = "joint"  # selection rule: "joint" or "descent"
 
 
 # The workloads the layer is exercised and measured on.
@@ -46,6 +47,9 @@ WORKLOADS = {
     "512k_k2048": Workload("512k_k2048", 1, 16, 524288, 64, "bf16", 4, 4, 2048, True),
     # the pages' best pyramid ablation (pooling factor 2) at the 98K length: S = 30720
     "98k_p2_k1536": Workload("98k_p2_k1536", 1, 16, 98304, 64, "bf16", 2, 3, 1536, True),
+    # the same budget chosen by hierarchical descent (k best per level, their children kept)
+    "98k_descent_k1536": Workload("98k_descent_k1536", 1, 16, 98304, 64, "bf16", 4, 3, 1536, True,
+                                  "descent"),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}

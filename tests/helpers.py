@@ -126,11 +126,11 @@ def assert_grad_close(got, exp, terms, dtype, what):
     return int((err > base).sum())
 
 
-def oracle_layer(Q, K, V, dO, p, L, k, dtype):
+def oracle_layer(Q, K, V, dO, p, L, k, dtype, rule="joint"):
     """Oracle forward (and backward when dO is given) of [B,H,N,d] tensors."""
     mode = MODE[dtype]
     Qn, Kn, Vn = np64(Q), np64(K), np64(V)
-    O, ctxs, sz = oracle.forward(Qn, Kn, Vn, p, L, k, mode)
+    O, ctxs, sz = oracle.forward(Qn, Kn, Vn, p, L, k, mode, rule=rule)
     grads = None
     if dO is not None:
         grads = oracle.backward(ctxs, np64(dO), sz, mode)

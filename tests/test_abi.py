@@ -37,7 +37,7 @@ def test_plan_struct_matches_binding():
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_plan_sizes_match_oracle(name):
     w = WORKLOADS[name]
-    p = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+    p = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype, select=w.select)
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     assert (p.S, p.M, p.Ntot, p.Ksel) == (sz.S, sz.M, sz.Ntot, sz.Ksel)
     assert list(p.raw.flat_off)[: w.L + 1] == sz.flat_off
@@ -67,6 +67,21 @@ def test_plan_validation(args, status):
     with pytest.raises(lh.LighthouseError) as e:
         lh.plan(*args)
     assert e.value.status == status
+
+
+def test_plan_descent_selection_option():
+    """The descent rule keeps the same S, adds its scratch to the top-K
+    workspace, and needs k <= N / p^(L-1)."""
+    joint = lh.plan(1, 2, 1024, 64, 4, 3, 64, "bf16")
+    desc = lh.plan(1, 2, 1024, 64, 4, 3, 64, "bf16", select="descent")  # n[2] = 64 = k
+    assert desc.S == joint.S and desc.raw.c.select == 1
+    assert desc.raw.topk_ws_bytes > joint.raw.topk_ws_bytes
+    with pytest.raises(lh.LighthouseError) as e:
+        lh.plan(1, 2, 1024, 64, 4, 3, 65, "bf16", select="descent")
+    assert e.value.status == lh.LH_ERR_INVALID_ARG
+    cfg = lh.LhConfig(1, 2, 1024, 64, 4, 3, 1, lh.LH_BF16, 7)
+    assert lh.LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(lh.LhPlan())) == lh.LH_ERR_INVALID_ARG
+    assert b"select" in lh.LIB.lh_last_error()
 
 
 def test_plan_rejects_unknown_dtype():

@@ -48,12 +48,13 @@ def _check(got, exp, terms, what):
                            f"max abs err {err.max():.3e}")
 
 
-@pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048", "98k_p2_k1536"])
+@pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048", "98k_p2_k1536",
+                                        "98k_descent_k1536"])
 def run(request):
     from long_context_hierarchical_b200 import lh
     w = WORKLOADS[request.param]
     Q, K, V, dO = make_workload_inputs(w, seed=0, device="cuda")
-    pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype)
+    pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype, select=w.select)
     O, ctx = lh.forward(pl, Q, K, V)
     grads = lh.backward(pl, dO, ctx) if request.param == "98k_k1536" else None
     pyr, scores = lh.pyramid_score(pl, Q, K, V)
@@ -71,7 +72,7 @@ def test_fullsize_selection_and_output(run, h):
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     Qh, Kh, Vh = (np64(run[x][0, h]) for x in ("Q", "K", "V"))
     # scores and selection, in full
-    cand, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz)
+    cand, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz, w.select)
     got_scores = np64(run["scores"][0, h])
     assert np.max(np.abs(got_scores - cand) / np.maximum(cand, 1e-30)) <= 1e-6
     assert np.array_equal(ctx.sel_idx[0, h].cpu().numpy(), sel_idx)
@@ -124,7 +125,7 @@ def test_fullsize_gradient_prefix(run):
     h = HEADS[1]
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     Qh, Kh, Vh, dOh = (np64(run[x][0, h]) for x in ("Q", "K", "V", "dO"))
-    _, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz)
+    _, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz, w.select)
     levels = [oracle.pyramid(X, sz, "bf16") for X in (Qh, Kh, Vh)]
     Qg, Kg, Vg = (oracle.gather(levels[t], sel_idx, sz) for t in range(3))
     Og_exact, lse = oracle.causal_attention(Qg, Kg, Vg)

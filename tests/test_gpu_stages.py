@@ -123,6 +123,56 @@ def test_topk_ties_and_random_scores(distinct):
         assert np.array_equal(inv[0, h].cpu().numpy(), ei)
 
 
+# (B, H, N, p, L, k, distinct score levels or None)
+DESCENT_CASES = {
+    "p4_L3": (1, 3, 4096, 4, 3, 40, None),
+    "p2_L4_ties": (1, 2, 1024, 2, 4, 16, 3),
+    "p2_L5": (1, 2, 2048, 2, 5, 8, None),
+    "p4_L2_ties": (1, 2, 512, 4, 2, 30, 2),
+    "k_is_n_coarsest": (1, 2, 1024, 4, 3, 64, None),
+    "all_equal": (1, 1, 1024, 2, 3, 20, 1),
+}
+
+
+@pytest.mark.parametrize("case", list(DESCENT_CASES))
+def test_descent_selection_on_seeded_scores(case):
+    """Hierarchical-descent selection (lh_select LH_SELECT_DESCENT) against
+    the oracle's rule, bit for bit, including ties everywhere."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k, distinct = DESCENT_CASES[case]
+    sz = oracle.sizes(N, p, L, k)
+    scores = make_scores(B, H, sz.M, seed=9, distinct=distinct)
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16", select="descent")
+    sel, inv = lh.topk(pl, scores.cuda())
+    for h in range(H):
+        mask = oracle.select_descent(scores[0, h].double().numpy(), sz)
+        es, ei = oracle.order_selection(mask, sz)
+        assert np.array_equal(sel[0, h].cpu().numpy(), es)
+        assert np.array_equal(inv[0, h].cpu().numpy(), ei)
+    lh.device_status()
+
+
+def test_descent_whole_layer():
+    """The whole layer with descent selection: selection bit-exact, output
+    and gradients within the attention tolerances."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k = 1, 2, 2048, 4, 3, 24
+    Q, K, V, dO = make_inputs(B, H, N, 64, "bf16", seed=4)
+    O_e, ctxs, sz, grads = oracle_layer(Q, K, V, dO, p, L, k, torch.bfloat16, rule="descent")
+    terms = grad_tolerance_terms(ctxs, grads, sz)
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16", select="descent")
+    dev = [x.cuda() for x in (Q, K, V, dO)]
+    O, ctx = lh.forward(pl, *dev[:3])
+    g = lh.backward(pl, dev[3], ctx)
+    torch.cuda.synchronize()
+    assert np.array_equal(ctx.sel_idx.cpu().numpy(), stack(ctxs, "sel_idx"))
+    assert np.array_equal(ctx.slot_of.cpu().numpy(), stack(ctxs, "slot_of"))
+    assert_grad_close(np64(O), O_e, terms["O"], torch.bfloat16, "O")
+    for got, i, key in ((g[0], 0, "dQ"), (g[1], 1, "dK"), (g[2], 2, "dV")):
+        assert_grad_close(np64(got), grads[i], terms[key], torch.bfloat16, key)
+    lh.device_status()
+
+
 def test_gather(case):
     c = case
     lh, pl, dt = c["lh"], c["pl"], c["dt"]
