@@ -7,7 +7,7 @@
  * gist.science "Long Context Pre-Training with Lighthouse Attention",
  * Technical Summary section 2).  Its four stages are
  *   1. a symmetric average-pool pyramid of Q, K and V       (lh_pyramid),
- *   2. parameter-free l2-norm scores and a joint top-K      (lh_score, lh_topk),
+ *   2. parameter-free l2-norm scores and a top-K selection  (lh_score, lh_topk),
  *   3. a gather into a causally ordered sub-sequence of length
  *      S = N/p^(L-1) + (L-1)*p*k and dense S x S causal attention
  *                                                            (lh_gather, lh_attn_fwd),
@@ -143,11 +143,14 @@ lh_status lh_pyramid_score(const lh_plan* plan, const void* Q, const void* K, co
                            lh_stream_t stream);
 
 /* Stage 2, selection and order (skill card "阶段 2", "阶段 3"; gist.science
- * 2.B-C).  From scores [B,H,M] selects, per (b,h), the Ksel largest by
- * (score desc, flat index asc), adds every level-(L-1) entry, and orders them
- * by (span end, level).  sel_idx: [B,H,S] int32 flat indices in gathered
- * order.  slot_of: [B,H,Ntot] int32, the slot of each pyramid entry or -1.
- * ws: plan->topk_ws_bytes of scratch (contents on entry are ignored). */
+ * 2.B-C).  From scores [B,H,M] selects, per (b,h), Ksel candidates by the
+ * plan's rule -- LH_SELECT_JOINT: the Ksel largest by (score desc, flat index
+ * asc); LH_SELECT_DESCENT: the p children of the k best entries of each
+ * level, from the coarsest down, a coarsest entry scoring the max of its p
+ * children -- adds every level-(L-1) entry, and orders them by (span end,
+ * level).  sel_idx: [B,H,S] int32 flat indices in gathered order.  slot_of:
+ * [B,H,Ntot] int32, the slot of each pyramid entry or -1.  ws:
+ * plan->topk_ws_bytes of scratch (contents on entry are ignored). */
 lh_status lh_topk(const lh_plan* plan, const float* scores, int32_t* sel_idx, int32_t* slot_of,
                   void* ws, size_t ws_bytes, lh_stream_t stream);
 
