@@ -84,6 +84,50 @@ def test_plan_descent_selection_option():
     assert b"select" in lh.LIB.lh_last_error()
 
 
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "lh.h"
+int main(void) {
+  lh_config c;
+  lh_plan p;
+  memset(&c, 0, sizeof c);
+  c.B = 1; c.H = 16; c.N = 98304; c.d = 64; c.p = 4; c.L = 3; c.k = 1536;
+  c.dtype = LH_BF16; c.select = LH_SELECT_JOINT;
+  if (lh_plan_bytes() != (int64_t)sizeof(lh_plan)) return 2;
+  if (lh_plan_init(&c, &p) != LH_OK) return 3;
+  c.k = 1 << 20;
+  if (lh_plan_init(&c, &p) != LH_ERR_INVALID_ARG) return 4;
+  printf("%lld %lld %s\n", (long long)p.S, (long long)p.M, lh_status_string(LH_ERR_TIMEOUT));
+  return 0;
+}
+"""
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    """A plain C11 program includes lh.h and calls the host-only entry points
+    of liblh.so (no GPU needed): the boundary is usable without PyTorch."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(lh.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        str(src), "-o", str(exe), "-L", libdir, "-llh", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    S, M, name = r.stdout.strip().split(maxsplit=2)
+    assert (int(S), int(M)) == (18432, 122880)
+    assert name == lh.LIB.lh_status_string(lh.LH_ERR_TIMEOUT).decode()
+
+
 def test_plan_rejects_unknown_dtype():
     cfg = lh.LhConfig(1, 2, 1024, 64, 4, 3, 1, 7)
     out = lh.LhPlan()
