@@ -104,6 +104,7 @@ class ClockSampler:
 STAGES = ("pyramid_score", "topk", "gather", "attn_fwd", "scatter",
           "scatter_bwd", "attn_bwd", "gather_bwd")
 # kernels each stage launches (lh_topk also issues one cudaMemsetAsync)
+# kernels per stage (top-K: 5 for the joint rule, 3 for the descent rule)
 LAUNCHES = {"pyramid_score": 1, "topk": 5, "gather": 1, "attn_fwd": 1, "scatter": 1,
             "scatter_bwd": 1, "attn_bwd": 2, "gather_bwd": 1}
 
@@ -466,7 +467,7 @@ def main():
                     "ms_per_step": e2e_ms,
                     "schedule": "lh.HostPipeline: step i's kernels overlap the copy-in of "
                                 "step i+1 and the copy-out of step i-1"},
-            "gpu_launches": sum(LAUNCHES.values()) * args.steps,
+            "gpu_launches": (sum(LAUNCHES.values()) - (2 if w.select == "descent" else 0)) * args.steps,
             "clocks": clk, "stages": stages, "extras": extras,
         }
         print(json.dumps(line), flush=True)
