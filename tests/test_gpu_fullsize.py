@@ -4,9 +4,10 @@ The layer runs on the GPU exactly as the benchmark runs it (lh_forward /
 lh_backward on the whole [1, 16, N, 64] problem).  The oracle then checks
 sampled heads: pyramid levels, scores and the selection in full; the
 attention output at sampled tokens (through the oracle's attention rows of
-the slots that reach them); and, at 98K with k = 1536, dQ/dK/dV on a
-4096-token prefix (oracle backward restricted to the slots that reach the
-prefix, with the full forward's LSE and D).
+the slots that reach them); and dQ/dK/dV on a 4096-token prefix (oracle
+backward restricted to the slots that reach the prefix, with the full
+forward's LSE and D), for every workload: 98K with k = 1536 and k = 6144,
+512K, 98K with p = 2, and 98K with the descent selection.
 """
 import numpy as np
 import pytest
@@ -56,7 +57,7 @@ def run(request):
     Q, K, V, dO = make_workload_inputs(w, seed=0, device="cuda")
     pl = lh.plan(w.B, w.H, w.N, w.d, w.p, w.L, w.k, w.dtype, select=w.select)
     O, ctx = lh.forward(pl, Q, K, V)
-    grads = lh.backward(pl, dO, ctx) if request.param == "98k_k1536" else None
+    grads = lh.backward(pl, dO, ctx)
     pyr, scores = lh.pyramid_score(pl, Q, K, V)
     torch.cuda.synchronize()
     lh.device_status()
@@ -118,9 +119,7 @@ def test_fullsize_selection_and_output(run, h):
 
 
 def test_fullsize_gradient_prefix(run):
-    """dQ, dK, dV on tokens t < 4096 of one head (98K, k = 1536)."""
-    if run["grads"] is None:
-        pytest.skip("gradients are checked on the 98K k=1536 workload")
+    """dQ, dK, dV on tokens t < 4096 of one head, every full-size workload."""
     w, ctx = run["w"], run["ctx"]
     h = HEADS[1]
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
