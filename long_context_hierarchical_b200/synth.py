@@ -34,7 +34,7 @@ class Workload:
     p: int
     L: int
     k: int
-    backward: bool
+    backward: bool  # the configuration the pages quote includes the backward pass
     select: str = "joint"  # selection rule: "joint" or "descent"
 
 
@@ -88,8 +88,10 @@ def make_inputs(B: int, H: int, N: int, d: int, dtype: str, seed: int = 0,
 
 
 def make_workload_inputs(w: Workload, seed: int = 0, device="cpu"):
-    return make_inputs(w.B, w.H, w.N, w.d, w.dtype, seed=seed, device=device,
-                       with_grad=w.backward)
+    """(Q, K, V, dO) of a workload.  dO is always drawn (after Q, K, V, so their
+    bytes do not depend on it): the benchmark times forward and backward of
+    every workload."""
+    return make_inputs(w.B, w.H, w.N, w.d, w.dtype, seed=seed, device=device, with_grad=True)
 
 
 def make_scores(B: int, H: int, M: int, seed: int = 0, distinct: int | None = None):
