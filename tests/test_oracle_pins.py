@@ -302,6 +302,19 @@ def test_descent_invariants_random(p, L, k, distinct):
         assert set(ranked[:k]) == set(parents.tolist())
 
 
+@pytest.mark.parametrize("p", [2, 4])
+def test_descent_and_joint_agree_when_everything_is_kept(p):
+    """L = 2 with k = N/p: both rules keep every entry of both levels, so the
+    gathered sub-sequence is the whole pyramid in (end, level) order."""
+    N = 16 * p
+    sz = lh.sizes(N, p, 2, N // p)
+    s0 = rng(5).random(N)
+    cand = lh.candidate_scores(s0, sz)
+    a, _ = lh.order_selection(lh.select(cand, sz), sz)
+    b, _ = lh.order_selection(lh.select_descent(cand, sz), sz)
+    assert np.array_equal(a, b) and a.size == sz.Ntot == sz.S
+
+
 def test_descent_needs_k_within_the_coarsest_level():
     sz = lh.sizes(64, 2, 4, 9)  # n_3 = 8 < k
     with pytest.raises(ValueError):
