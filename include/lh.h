@@ -120,7 +120,8 @@ typedef struct {
  * LH_ERR_INVALID_ARG when the method itself is undefined for the config
  * (N % p^(L-1) != 0, L < 1, p < 2, k < 0, (L-1)*p*k > M, S >= 2^31, an
  * unknown select, descent with k > n[L-1]) and LH_ERR_UNSUPPORTED for
- * shapes this build does not implement. */
+ * shapes this build does not implement (d != 64, p not in {2, 4}, L > 5,
+ * p^(L-1) > 256, B*H > 65535, bf16 with B*H*S >= 2^31). */
 lh_status lh_plan_init(const lh_config* cfg, lh_plan* out);
 
 /* Stage 1 (skill card "阶段 1"; gist.science 2.A).  Writes pyramid levels

@@ -136,6 +136,11 @@ lh_status lh_plan_init(const lh_config* cfg, lh_plan* out) {
     return fail(LH_ERR_INVALID_ARG, "descent selection needs k <= N / p^(L-1)");
   if (p.S >= (int64_t(1) << 31) || p.Ntot >= (int64_t(1) << 31))
     return fail(LH_ERR_INVALID_ARG, "S and the pyramid size must stay below 2^31");
+  // The per-head stage kernels put the head on the grid's y dimension.
+  if ((int64_t)c.B * c.H > 65535) return fail(LH_ERR_UNSUPPORTED, "B * H above 65535 is not built");
+  // The bf16 attention addresses rows of [B*H*S, d] with 32-bit TMA coordinates.
+  if (c.dtype == LH_BF16 && (int64_t)c.B * c.H * p.S >= (int64_t(1) << 31))
+    return fail(LH_ERR_UNSUPPORTED, "bf16 attention needs B * H * S < 2^31 (TMA row coordinates)");
   p.elem_bytes = c.dtype == LH_BF16 ? 2 : 4;
 
   const int64_t BH = (int64_t)c.B * c.H;

@@ -59,6 +59,11 @@ def test_plan_sizes_match_oracle(name):
     ((1, 2, 1152, 64, 3, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # p = 3
     ((1, 2, 4096, 64, 2, 6, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # L = 6
     ((1, 2, 4096, 64, 4, 5, 1, "bf16"), None),                     # p^(L-1) = 256: built
+    ((1, 65536, 64, 64, 4, 2, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),  # B*H above the grid's y limit
+    ((3, 21845, 64, 64, 4, 2, 1, "bf16"), None),                   # B*H = 65535: built
+    ((1, 2048, 2**20, 64, 4, 1, 0, "bf16"), lh.LH_ERR_UNSUPPORTED),  # B*H*S = 2^31: TMA rows
+    ((1, 2047, 2**20, 64, 4, 1, 0, "bf16"), None),                   # B*H*S < 2^31: built
+    ((1, 2048, 2**20, 64, 4, 1, 0, "f32"), None),                    # fp32 has no TMA limit
 ])
 def test_plan_validation(args, status):
     if status is None:
