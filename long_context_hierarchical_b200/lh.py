@@ -120,6 +120,49 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(t, name: str, dtype, numel: int):
+    """Check a tensor the library will read or write as ``numel`` contiguous
+    elements of ``dtype`` in device memory (the C ABI sees only its pointer)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, the call needs {numel}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor (got {t.device})")
+
+
+def _require_tokens(pl, **tensors):
+    """[B,H,N,d] tensors of the plan's dtype."""
+    c = pl.raw.c
+    for name, t in tensors.items():
+        _require(t, name, pl.dtype, c.B * c.H * c.N * c.d)
+
+
+def _require_rows(pl, **tensors):
+    """[B,H,S,d] gathered tensors of the plan's dtype."""
+    c = pl.raw.c
+    for name, t in tensors.items():
+        _require(t, name, pl.dtype, c.B * c.H * pl.S * c.d)
+
+
+def _attn_shape(Qg, **others):
+    """(BH, S, d) of [..., S, d] attention operands; every other operand has
+    Qg's dtype and size."""
+    if not isinstance(Qg, torch.Tensor) or Qg.dim() < 2:
+        raise ValueError("Qg: expected a tensor of shape [..., S, d]")
+    if Qg.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"Qg: dtype {Qg.dtype}, expected torch.bfloat16 or torch.float32")
+    S, d = Qg.shape[-2], Qg.shape[-1]
+    _require(Qg, "Qg", Qg.dtype, Qg.numel())
+    for name, t in others.items():
+        _require(t, name, Qg.dtype, Qg.numel())
+    return Qg.numel() // max(S * d, 1), S, d
+
+
 def _stream(stream=None):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -186,6 +229,7 @@ def _bytes(n, device):
 
 def pyramid_score(pl: Plan, Q, K, V, stream=None):
     """Levels 1..L-1 of Q, K, V ([B,H,Npyr,d] each) and candidate scores [B,H,M]."""
+    _require_tokens(pl, Q=Q, K=K, V=V)
     c = pl.raw.c
     dev = Q.device
     pyr = [_empty((c.B, c.H, max(pl.Npyr, 1), c.d), Q.dtype, dev) for _ in range(3)]
@@ -196,6 +240,7 @@ def pyramid_score(pl: Plan, Q, K, V, stream=None):
 
 
 def pyramid(pl: Plan, Q, K, V, stream=None):
+    _require_tokens(pl, Q=Q, K=K, V=V)
     c = pl.raw.c
     pyr = [_empty((c.B, c.H, max(pl.Npyr, 1), c.d), Q.dtype, Q.device) for _ in range(3)]
     _check(LIB.lh_pyramid(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), *map(_ptr, pyr),
@@ -204,6 +249,7 @@ def pyramid(pl: Plan, Q, K, V, stream=None):
 
 
 def score(pl: Plan, Q, K, stream=None):
+    _require_tokens(pl, Q=Q, K=K)
     c = pl.raw.c
     scores = _empty((c.B, c.H, max(pl.M, 1)), torch.float32, Q.device)
     _check(LIB.lh_score(pl.byref(), _ptr(Q), _ptr(K), _ptr(scores), _stream(stream)), "lh_score")
@@ -213,6 +259,7 @@ def score(pl: Plan, Q, K, stream=None):
 def topk(pl: Plan, scores, stream=None):
     """(sel_idx [B,H,S] int32, slot_of [B,H,Ntot] int32) from scores [B,H,M]."""
     c = pl.raw.c
+    _require(scores, "scores", torch.float32, c.B * c.H * pl.M)
     dev = scores.device
     sel = _empty((c.B, c.H, pl.S), torch.int32, dev)
     inv = _empty((c.B, c.H, pl.Ntot), torch.int32, dev)
@@ -223,7 +270,13 @@ def topk(pl: Plan, scores, stream=None):
 
 
 def gather(pl: Plan, Q, K, V, pyr, sel_idx, stream=None):
+    _require_tokens(pl, Q=Q, K=K, V=V)
     c = pl.raw.c
+    if len(pyr) != 3:
+        raise ValueError("pyr: expected the three pyramids (Q, K, V)")
+    for name, t in zip(("pyrQ", "pyrK", "pyrV"), pyr):
+        _require(t, name, pl.dtype, c.B * c.H * pl.Npyr * c.d)
+    _require(sel_idx, "sel_idx", torch.int32, c.B * c.H * pl.S)
     out = [_empty((c.B, c.H, pl.S, c.d), Q.dtype, Q.device) for _ in range(3)]
     _check(LIB.lh_gather(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), *map(_ptr, pyr), _ptr(sel_idx),
                          *map(_ptr, out), _stream(stream)), "lh_gather")
@@ -236,8 +289,7 @@ def _dtype_code(t):
 
 def attn_fwd(Qg, Kg, Vg, stream=None):
     """Causal attention on [..., S, d] tensors: (O, lse[..., S] natural log)."""
-    S, d = Qg.shape[-2], Qg.shape[-1]
-    BH = Qg.numel() // (S * d)
+    BH, S, d = _attn_shape(Qg, Kg=Kg, Vg=Vg)
     O = torch.empty_like(Qg)
     lse = _empty(Qg.shape[:-1], torch.float32, Qg.device)
     _check(LIB.lh_attn_fwd(BH, S, d, _dtype_code(Qg), _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(O),
@@ -246,8 +298,10 @@ def attn_fwd(Qg, Kg, Vg, stream=None):
 
 
 def attn_bwd(Qg, Kg, Vg, Og, lse, dOg, D=None, stream=None):
-    S, d = Qg.shape[-2], Qg.shape[-1]
-    BH = Qg.numel() // (S * d)
+    BH, S, d = _attn_shape(Qg, Kg=Kg, Vg=Vg, Og=Og, dOg=dOg)
+    _require(lse, "lse", torch.float32, BH * S)
+    if D is not None:
+        _require(D, "D", torch.float32, BH * S)
     code = _dtype_code(Qg)
     dQ, dK, dV = torch.empty_like(Qg), torch.empty_like(Kg), torch.empty_like(Vg)
     ws = _bytes(LIB.lh_attn_bwd_ws_bytes(BH, S, d, code), Qg.device)
@@ -260,8 +314,8 @@ def attn_bwd(Qg, Kg, Vg, Og, lse, dOg, D=None, stream=None):
 def attn_bwd_static(Qg, Kg, Vg, Og, lse, dOg, stream=None):
     """lh_attn_bwd with D computed into the library's own scratch array
     (no workspace: for callers that cannot allocate device memory)."""
-    S, d = Qg.shape[-2], Qg.shape[-1]
-    BH = Qg.numel() // (S * d)
+    BH, S, d = _attn_shape(Qg, Kg=Kg, Vg=Vg, Og=Og, dOg=dOg)
+    _require(lse, "lse", torch.float32, BH * S)
     dQ, dK, dV = torch.empty_like(Qg), torch.empty_like(Kg), torch.empty_like(Vg)
     _check(LIB.lh_attn_bwd_static(BH, S, d, _dtype_code(Qg), _ptr(Qg), _ptr(Kg), _ptr(Vg), _ptr(Og),
                                   _ptr(lse), _ptr(dOg), _ptr(dQ), _ptr(dK), _ptr(dV),
@@ -270,7 +324,9 @@ def attn_bwd_static(Qg, Kg, Vg, Og, lse, dOg, stream=None):
 
 
 def scatter(pl: Plan, Og, slot_of, stream=None):
+    _require_rows(pl, Og=Og)
     c = pl.raw.c
+    _require(slot_of, "slot_of", torch.int32, c.B * c.H * pl.Ntot)
     O = _empty((c.B, c.H, c.N, c.d), Og.dtype, Og.device)
     _check(LIB.lh_scatter(pl.byref(), _ptr(Og), _ptr(slot_of), _ptr(O), _stream(stream)),
            "lh_scatter")
@@ -278,7 +334,10 @@ def scatter(pl: Plan, Og, slot_of, stream=None):
 
 
 def scatter_bwd(pl: Plan, dO, Og, sel_idx, stream=None):
+    _require_tokens(pl, dO=dO)
+    _require_rows(pl, Og=Og)
     c = pl.raw.c
+    _require(sel_idx, "sel_idx", torch.int32, c.B * c.H * pl.S)
     dOg = _empty((c.B, c.H, pl.S, c.d), dO.dtype, dO.device)
     D = _empty((c.B, c.H, pl.S), torch.float32, dO.device)
     _check(LIB.lh_scatter_bwd(pl.byref(), _ptr(dO), _ptr(Og), _ptr(sel_idx), _ptr(dOg), _ptr(D),
@@ -287,7 +346,9 @@ def scatter_bwd(pl: Plan, dO, Og, sel_idx, stream=None):
 
 
 def gather_bwd(pl: Plan, dQg, dKg, dVg, slot_of, stream=None):
+    _require_rows(pl, dQg=dQg, dKg=dKg, dVg=dVg)
     c = pl.raw.c
+    _require(slot_of, "slot_of", torch.int32, c.B * c.H * pl.Ntot)
     out = [_empty((c.B, c.H, c.N, c.d), dQg.dtype, dQg.device) for _ in range(3)]
     _check(LIB.lh_gather_bwd(pl.byref(), _ptr(dQg), _ptr(dKg), _ptr(dVg), _ptr(slot_of),
                              *map(_ptr, out), _stream(stream)), "lh_gather_bwd")
@@ -340,6 +401,7 @@ class Workspace:
 def forward(pl: Plan, Q, K, V, O=None, ctx: Context | None = None, ws: Workspace | None = None,
             stream=None):
     """O = Lighthouse(Q, K, V); returns (O, ctx)."""
+    _require_tokens(pl, Q=Q, K=K, V=V)
     dev = Q.device
     if O is None:
         O = torch.empty_like(Q)
@@ -347,6 +409,9 @@ def forward(pl: Plan, Q, K, V, O=None, ctx: Context | None = None, ws: Workspace
         ctx = Context(pl, dev)
     if ws is None:
         ws = Workspace(pl, dev)
+    _require_tokens(pl, O=O)
+    _require(ctx.buf, "ctx", torch.uint8, pl.raw.ctx_bytes)
+    _require(ws.buf, "ws", torch.uint8, pl.raw.ws_bytes)
     _check(LIB.lh_forward(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(ctx.buf),
                           _ptr(ws.buf), _stream(stream)), "lh_forward")
     return O, ctx
@@ -355,10 +420,14 @@ def forward(pl: Plan, Q, K, V, O=None, ctx: Context | None = None, ws: Workspace
 def backward(pl: Plan, dO, ctx: Context, dQ=None, dK=None, dV=None, ws: Workspace | None = None,
              stream=None):
     """(dQ, dK, dV) from dO and the ctx of the matching forward."""
+    _require_tokens(pl, dO=dO)
     if dQ is None:
         dQ, dK, dV = torch.empty_like(dO), torch.empty_like(dO), torch.empty_like(dO)
     if ws is None:
         ws = Workspace(pl, dO.device)
+    _require_tokens(pl, dQ=dQ, dK=dK, dV=dV)
+    _require(ctx.buf, "ctx", torch.uint8, pl.raw.ctx_bytes)
+    _require(ws.buf, "ws", torch.uint8, pl.raw.ws_bytes)
     _check(LIB.lh_backward(pl.byref(), _ptr(dO), _ptr(ctx.buf), _ptr(dQ), _ptr(dK), _ptr(dV),
                            _ptr(ws.buf), _stream(stream)), "lh_backward")
     return dQ, dK, dV

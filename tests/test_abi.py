@@ -165,3 +165,32 @@ def test_entry_points_reject_bad_pointers_before_launching():
 def test_status_strings():
     for s in range(6):
         assert lh.LIB.lh_status_string(s)
+
+
+def test_binding_checks_tensor_arguments_before_calling_the_library():
+    """The binding refuses a tensor of the wrong dtype, layout, size or device
+    before any pointer reaches the library (a kernel would read or write past
+    it)."""
+    import torch
+    pl = lh.plan(1, 2, 256, 64, 4, 3, 4, "bf16")
+    tok = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    cases = [
+        (lambda: lh.forward(pl, tok.float(), tok, tok), "dtype"),
+        (lambda: lh.forward(pl, tok.transpose(2, 3), tok, tok), "contiguous"),
+        (lambda: lh.forward(pl, tok[:, :1], tok, tok), "elements"),
+        (lambda: lh.forward(pl, tok, tok, tok), "CUDA"),
+        (lambda: lh.topk(pl, torch.zeros(1, 2, pl.M, dtype=torch.float64)), "dtype"),
+        (lambda: lh.scatter(pl, torch.zeros(1, 2, pl.S, 64),
+                            torch.zeros(1, 2, pl.Ntot, dtype=torch.int32)), "dtype"),
+        (lambda: lh.gather_bwd(pl, *(torch.zeros(1, 2, pl.S - 1, 64, dtype=torch.bfloat16),) * 3,
+                               torch.zeros(1, 2, pl.Ntot, dtype=torch.int32)), "elements"),
+        (lambda: lh.attn_fwd(*(torch.zeros(2, 128, 64, dtype=torch.float16),) * 3), "dtype"),
+        (lambda: lh.attn_fwd(torch.zeros(2, 128, 64).transpose(1, 2), None, None), "contiguous"),
+        (lambda: lh.attn_bwd(torch.zeros(64), None, None, None, None, None), "[..., S, d]"),
+        (lambda: lh.attn_fwd(*(torch.zeros(2, 128, 64),) * 3), "CUDA"),
+        (lambda: lh.backward(pl, [0.0], None), "torch.Tensor"),
+    ]
+    for call, what in cases:
+        with pytest.raises((ValueError, TypeError)) as e:
+            call()
+        assert what in str(e.value), (what, str(e.value))
