@@ -251,6 +251,14 @@ lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void
  * reset != 0 clears the word. */
 lh_status lh_device_status(int reset);
 
+/* Self-test of that failure path: enqueues one CTA that waits, through the
+ * same bounded mbarrier wait as the attention kernels, on a barrier nothing
+ * signals.  The wait gives up after its budget (about 2 s at full SM clock),
+ * the kernel returns normally and the next lh_device_status reports
+ * LH_ERR_TIMEOUT; the CUDA context stays usable.  Returns LH_ERR_CUDA only if
+ * the launch fails. */
+lh_status lh_selftest_wait_timeout(lh_stream_t stream);
+
 const char* lh_status_string(lh_status s);
 const char* lh_last_error(void);
 

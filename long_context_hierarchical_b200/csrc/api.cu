@@ -401,6 +401,11 @@ lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void
   return ok();
 }
 
+lh_status lh_selftest_wait_timeout(lh_stream_t stream) {
+  LH_TRY(cuda_status(launch_wait_timeout_selftest(as_cuda(stream)), "lh_selftest_wait_timeout"));
+  return ok();
+}
+
 lh_status lh_device_status(int reset) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e, "lh_device_status");

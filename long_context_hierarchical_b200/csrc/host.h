@@ -49,5 +49,7 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, co
                             const void* Vg, const void* Og, const float* lse, const void* dOg,
                             const float* D, void* dQg, void* dKg, void* dVg, void* ws,
                             cudaStream_t st);
+// One CTA waiting on a barrier nothing signals (the failure-path self-test).
+cudaError_t launch_wait_timeout_selftest(cudaStream_t st);
 
 }  // namespace lh

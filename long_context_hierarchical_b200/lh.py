@@ -29,6 +29,7 @@ EXPORTS = (
     "lh_attn_fwd", "lh_attn_bwd_ws_bytes", "lh_attn_bwd", "lh_scatter", "lh_scatter_bwd",
     "lh_gather_bwd", "lh_forward", "lh_backward", "lh_device_status", "lh_status_string",
     "lh_last_error", "lh_plan_bytes", "lh_attn_bwd_static", "lh_set_deterministic",
+    "lh_selftest_wait_timeout",
 )
 
 
@@ -86,6 +87,7 @@ def _load():
         "lh_forward": (PLAN, P, P, P, P, P, P, P),
         "lh_backward": (PLAN, P, P, P, P, P, P, P),
         "lh_device_status": (ctypes.c_int,),
+        "lh_selftest_wait_timeout": (P,),
         "lh_attn_bwd_static": (I64, I64, I32, I32, P, P, P, P, P, P, P, P, P, P),
     }
     for name, args in sig.items():
@@ -507,6 +509,12 @@ def set_deterministic(on: bool):
     """Process-wide: bit-reproducible bf16 attention backward (two kernels, no
     atomics) for lh_attn_bwd / lh_backward calls enqueued afterwards."""
     LIB.lh_set_deterministic(1 if on else 0)
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the failure-path self-test (a bounded wait that must give up);
+    the next device_status() raises LighthouseError with LH_ERR_TIMEOUT."""
+    _check(LIB.lh_selftest_wait_timeout(_stream(stream)), "lh_selftest_wait_timeout")
 
 
 def device_status(reset: bool = True):

@@ -2,9 +2,10 @@
 
 Some callers hold only their inputs and outputs and cannot allocate device
 memory; lh_attn_bwd_static serves them by keeping its scratch (the row term D)
-in a fixed array inside the library.  This file is collected last so that a
-run stopping at the first failure has run every other test before it; it
-passes alone in a fresh process and after the rest of the suite.
+in a fixed array inside the library.  This file is collected after the stage
+and whole-layer tests so that a run stopping at the first failure has run
+them before it; it passes alone in a fresh process and after the rest of the
+suite.
 """
 import ctypes
 
