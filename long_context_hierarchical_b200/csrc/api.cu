@@ -1,6 +1,7 @@
 // C-ABI entry points of the Lighthouse layer: validation, buffer layout and
 // the stage order of the whole forward and backward pass.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdio.h>
 
 #include <string>
@@ -8,6 +9,15 @@
 #include "host.h"
 
 namespace lh {
+
+// NVTX range over one entry point or stage (a no-op unless a profiler is
+// attached), so a trace shows the stages by name around their launches.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 // Device status word (LH_OK or LH_ERR_TIMEOUT); kernels with bounded waits
 // receive its address from device_status_ptr().
@@ -203,6 +213,7 @@ static lh_status check_plan(const lh_plan* plan) {
 
 lh_status lh_pyramid(const lh_plan* plan, const void* Q, const void* K, const void* V,
                      void* pyrQ, void* pyrK, void* pyrV, lh_stream_t stream) {
+  Range range("lh_pyramid");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K); LH_CHECK_PTR(V);
   if (plan->Npyr > 0) { LH_CHECK_PTR(pyrQ); LH_CHECK_PTR(pyrK); LH_CHECK_PTR(pyrV); }
@@ -214,6 +225,7 @@ lh_status lh_pyramid(const lh_plan* plan, const void* Q, const void* K, const vo
 
 lh_status lh_score(const lh_plan* plan, const void* Q, const void* K, float* scores,
                    lh_stream_t stream) {
+  Range range("lh_score");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K);
   if (plan->M == 0) return ok();
@@ -226,6 +238,7 @@ lh_status lh_score(const lh_plan* plan, const void* Q, const void* K, float* sco
 lh_status lh_pyramid_score(const lh_plan* plan, const void* Q, const void* K, const void* V,
                            void* pyrQ, void* pyrK, void* pyrV, float* scores,
                            lh_stream_t stream) {
+  Range range("lh_pyramid_score");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K); LH_CHECK_PTR(V);
   if (plan->Npyr > 0) { LH_CHECK_PTR(pyrQ); LH_CHECK_PTR(pyrK); LH_CHECK_PTR(pyrV); }
@@ -239,6 +252,7 @@ lh_status lh_pyramid_score(const lh_plan* plan, const void* Q, const void* K, co
 
 lh_status lh_topk(const lh_plan* plan, const float* scores, int32_t* sel_idx, int32_t* slot_of,
                   void* ws, size_t ws_bytes, lh_stream_t stream) {
+  Range range("lh_topk");
   LH_TRY(check_plan(plan));
   if (plan->M > 0) LH_CHECK_PTR(scores);
   LH_CHECK_PTR(sel_idx); LH_CHECK_PTR(slot_of);
@@ -254,6 +268,7 @@ lh_status lh_topk(const lh_plan* plan, const float* scores, int32_t* sel_idx, in
 lh_status lh_gather(const lh_plan* plan, const void* Q, const void* K, const void* V,
                     const void* pyrQ, const void* pyrK, const void* pyrV,
                     const int32_t* sel_idx, void* Qg, void* Kg, void* Vg, lh_stream_t stream) {
+  Range range("lh_gather");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K); LH_CHECK_PTR(V); LH_CHECK_PTR(sel_idx);
   if (plan->Npyr > 0) { LH_CHECK_PTR(pyrQ); LH_CHECK_PTR(pyrK); LH_CHECK_PTR(pyrV); }
@@ -275,6 +290,7 @@ static lh_status check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
 
 lh_status lh_attn_fwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, void* Og, float* lse, lh_stream_t stream) {
+  Range range("lh_attn_fwd");
   LH_TRY(check_attn(BH, S, d, dtype));
   LH_CHECK_PTR(Qg); LH_CHECK_PTR(Kg); LH_CHECK_PTR(Vg); LH_CHECK_PTR(Og); LH_CHECK_PTR(lse);
   LH_TRY(cuda_status(launch_attn_fwd(BH, S, dtype, Qg, Kg, Vg, Og, lse, as_cuda(stream)),
@@ -293,6 +309,7 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
                       const void* Kg, const void* Vg, const void* Og, const float* lse,
                       const void* dOg, const float* D, void* dQg, void* dKg, void* dVg,
                       void* ws, size_t ws_bytes, lh_stream_t stream) {
+  Range range("lh_attn_bwd");
   LH_TRY(check_attn(BH, S, d, dtype));
   LH_CHECK_PTR(Qg); LH_CHECK_PTR(Kg); LH_CHECK_PTR(Vg); LH_CHECK_PTR(lse); LH_CHECK_PTR(dOg);
   LH_CHECK_PTR(dQg); LH_CHECK_PTR(dKg); LH_CHECK_PTR(dVg);
@@ -311,6 +328,7 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
 
 lh_status lh_scatter(const lh_plan* plan, const void* Og, const int32_t* slot_of, void* O,
                      lh_stream_t stream) {
+  Range range("lh_scatter");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Og); LH_CHECK_PTR(slot_of); LH_CHECK_PTR(O);
   LH_TRY(cuda_status(launch_scatter(*plan, Og, slot_of, O, as_cuda(stream)), "lh_scatter"));
@@ -319,6 +337,7 @@ lh_status lh_scatter(const lh_plan* plan, const void* Og, const int32_t* slot_of
 
 lh_status lh_scatter_bwd(const lh_plan* plan, const void* dO, const void* Og,
                          const int32_t* sel_idx, void* dOg, float* D, lh_stream_t stream) {
+  Range range("lh_scatter_bwd");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(dO); LH_CHECK_PTR(Og); LH_CHECK_PTR(sel_idx); LH_CHECK_PTR(dOg); LH_CHECK_PTR(D);
   LH_TRY(cuda_status(launch_scatter_bwd(*plan, dO, Og, sel_idx, dOg, D, as_cuda(stream)),
@@ -328,6 +347,7 @@ lh_status lh_scatter_bwd(const lh_plan* plan, const void* dO, const void* Og,
 
 lh_status lh_gather_bwd(const lh_plan* plan, const void* dQg, const void* dKg, const void* dVg,
                         const int32_t* slot_of, void* dQ, void* dK, void* dV, lh_stream_t stream) {
+  Range range("lh_gather_bwd");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(dQg); LH_CHECK_PTR(dKg); LH_CHECK_PTR(dVg); LH_CHECK_PTR(slot_of);
   LH_CHECK_PTR(dQ); LH_CHECK_PTR(dK); LH_CHECK_PTR(dV);
@@ -338,6 +358,7 @@ lh_status lh_gather_bwd(const lh_plan* plan, const void* dQg, const void* dKg, c
 
 lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const void* V, void* O,
                      void* ctx, void* ws, lh_stream_t stream) {
+  Range range("lh_forward");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K); LH_CHECK_PTR(V); LH_CHECK_PTR(O);
   LH_CHECK_PTR(ctx); LH_CHECK_PTR(ws);
@@ -358,20 +379,35 @@ lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const vo
   void* tws = w + plan->ws_topk;
   const int64_t BH = (int64_t)plan->c.B * plan->c.H;
 
-  if (plan->Npyr > 0 || plan->M > 0)
+  if (plan->Npyr > 0 || plan->M > 0) {
+    Range r("pyramid_score");
     LH_TRY(cuda_status(launch_pyramid_score(*plan, Q, K, V, pyrQ, pyrK, pyrV, scores,
                                             plan->Npyr > 0, plan->M > 0, st), "lh_forward/pyramid"));
-  LH_TRY(cuda_status(launch_topk(*plan, scores, sel_idx, slot_of, tws, st), "lh_forward/topk"));
-  LH_TRY(cuda_status(launch_gather(*plan, Q, K, V, pyrQ, pyrK, pyrV, sel_idx, Qg, Kg, Vg, st),
-                     "lh_forward/gather"));
-  LH_TRY(cuda_status(launch_attn_fwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, st),
-                     "lh_forward/attention"));
-  LH_TRY(cuda_status(launch_scatter(*plan, Og, slot_of, O, st), "lh_forward/scatter"));
+  }
+  {
+    Range r("topk");
+    LH_TRY(cuda_status(launch_topk(*plan, scores, sel_idx, slot_of, tws, st), "lh_forward/topk"));
+  }
+  {
+    Range r("gather");
+    LH_TRY(cuda_status(launch_gather(*plan, Q, K, V, pyrQ, pyrK, pyrV, sel_idx, Qg, Kg, Vg, st),
+                       "lh_forward/gather"));
+  }
+  {
+    Range r("attn_fwd");
+    LH_TRY(cuda_status(launch_attn_fwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, st),
+                       "lh_forward/attention"));
+  }
+  {
+    Range r("scatter");
+    LH_TRY(cuda_status(launch_scatter(*plan, Og, slot_of, O, st), "lh_forward/scatter"));
+  }
   return ok();
 }
 
 lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void* dQ, void* dK,
                       void* dV, void* ws, lh_stream_t stream) {
+  Range range("lh_backward");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(dO); LH_CHECK_PTR(ctx); LH_CHECK_PTR(dQ); LH_CHECK_PTR(dK); LH_CHECK_PTR(dV);
   LH_CHECK_PTR(ws);
@@ -393,11 +429,20 @@ lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void
   void* aws = w + plan->ws_attn;
   const int64_t BH = (int64_t)plan->c.B * plan->c.H;
 
-  LH_TRY(cuda_status(launch_scatter_bwd(*plan, dO, Og, sel_idx, dOg, D, st), "lh_backward/scatter"));
-  LH_TRY(cuda_status(launch_attn_bwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg,
-                                     dKg, dVg, aws, st), "lh_backward/attention"));
-  LH_TRY(cuda_status(launch_gather_bwd(*plan, dQg, dKg, dVg, slot_of, dQ, dK, dV, st),
-                     "lh_backward/gather"));
+  {
+    Range r("scatter_bwd");
+    LH_TRY(cuda_status(launch_scatter_bwd(*plan, dO, Og, sel_idx, dOg, D, st), "lh_backward/scatter"));
+  }
+  {
+    Range r("attn_bwd");
+    LH_TRY(cuda_status(launch_attn_bwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg,
+                                       dKg, dVg, aws, st), "lh_backward/attention"));
+  }
+  {
+    Range r("gather_bwd");
+    LH_TRY(cuda_status(launch_gather_bwd(*plan, dQg, dKg, dVg, slot_of, dQ, dK, dV, st),
+                       "lh_backward/gather"));
+  }
   return ok();
 }
 
