@@ -69,7 +69,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// 2-D TMA tile load (no multicast) completing on an mbarrier.
+// 2-D TMA tile load into this CTA's own shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
   asm volatile(
@@ -79,8 +79,8 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 2-D TMA reduce-add of a shared-memory box into global memory (no
-// multicast), tracked by this thread's bulk async-group.
+// 2-D TMA reduce-add of a shared-memory box of this CTA into global memory,
+// tracked by this thread's bulk async-group.
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
   asm volatile(
       "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
