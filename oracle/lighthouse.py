@@ -384,6 +384,36 @@ def causal_attention_bwd(Qg, Kg, Vg, dOg, lse, D):
     return dQ, dK, dV
 
 
+def attention_bwd_rows(Qg, Kg, Vg, dOg, lse, D, q_rows, k_cols):
+    """The gradients of ``causal_attention_bwd`` for some rows only.
+
+    dQg of query row r needs the keys j <= r only; dKg and dVg of key
+    column c need every query row i >= c, with that row's forward LSE and
+    D_i, which the caller passes for all S rows.  Each row and column is
+    formed on its own, straight from the definitions: P_ij = exp(s_ij -
+    lse_i), dP_ij = dOg_i . Vg_j, dS_ij = P_ij (dP_ij - D_i), dQg_r =
+    sum_j dS_rj Kg_j / sqrt(d), dKg_c = sum_i dS_ic Qg_i / sqrt(d), dVg_c =
+    sum_i P_ic dOg_i.  Returns (dQg[q_rows], dKg[k_cols], dVg[k_cols]).
+    """
+    S, d = Qg.shape
+    scale = 1.0 / np.sqrt(d)
+    q_rows = np.asarray(q_rows, dtype=np.int64)
+    k_cols = np.asarray(k_cols, dtype=np.int64)
+    dQ = np.empty((q_rows.size, d), dtype=np.float64)
+    for a, r in enumerate(q_rows):
+        P = np.exp((Kg[: r + 1] @ Qg[r]) * scale - lse[r])
+        dS = P * (Vg[: r + 1] @ dOg[r] - D[r])
+        dQ[a] = (dS @ Kg[: r + 1]) * scale
+    dK = np.empty((k_cols.size, d), dtype=np.float64)
+    dV = np.empty((k_cols.size, Vg.shape[1]), dtype=np.float64)
+    for a, c in enumerate(k_cols):
+        P = np.exp((Qg[c:] @ Kg[c]) * scale - lse[c:])
+        dS = P * (dOg[c:] @ Vg[c] - D[c:])
+        dK[a] = (dS @ Qg[c:]) * scale
+        dV[a] = P @ dOg[c:]
+    return dQ, dK, dV
+
+
 def gather_bwd(dXg, slot_of, sz: Sizes, mode: str):
     """Adjoint of pyramid + gather: dX[t] = sum_l dXg[slot(l, t // p^l)] / p^l.
 

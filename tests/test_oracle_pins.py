@@ -450,6 +450,89 @@ def test_finite_difference_gradients():
             assert abs(fd - grad[t, c]) <= 1e-6 * max(1.0, abs(fd)), (name, t, c, fd, grad[t, c])
 
 
+def test_attention_bwd_rows_equals_the_full_backward():
+    """The restricted backward (some dQg rows, some dKg / dVg rows) equals the
+    same rows of the full one, which finite differences and torch autograd
+    pin (test_finite_difference_gradients, test_L1_is_dense_causal_sdpa)."""
+    S, d = 600, 16
+    Q, K, V = rand_head(S, d, 11), rand_head(S, d, 12), rand_head(S, d, 13)
+    dO = rand_head(S, d, 14, scale=False)
+    O, lse = lh.causal_attention(Q, K, V)
+    D = np.sum(dO * O, axis=1)
+    fq, fk, fv = lh.causal_attention_bwd(Q, K, V, dO, lse, D)
+    rows, cols = [0, 1, 127, 128, 300, 511, 512, 599], [0, 5, 127, 128, 450, 598, 599]
+    q, k, v = lh.attention_bwd_rows(Q, K, V, dO, lse, D, rows, cols)
+    for got, full, idx in ((q, fq, rows), (k, fk, cols), (v, fv, cols)):
+        ref = full[idx]
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def _rounding_case(d=8, seed=3):
+    """The hand-worked selection case (N=8, p=2, L=3, k=1) with inputs that
+    give exactly its level-0 scores: K_t has norm 5/8 (a 3-4-5 direction that
+    changes from token to token) and Q_t = (s0[t] - 5/8) e_0, all values exact
+    in bf16; V and dO are seeded bf16 values."""
+    g = GOLDEN["select_order_scatter"]
+    N = g["N"]
+    s0 = np.array(g["s0"], float)
+    dirs = [(3, 4), (4, 3), (-3, 4), (4, -3), (-4, -3), (-3, -4), (3, -4), (-4, 3)]
+    K = np.zeros((N, d))
+    K[:, :2] = np.array(dirs, float) / 8
+    Q = np.zeros((N, d))
+    Q[:, 0] = s0 - 0.625
+    r = rng(seed)
+    V = lh.round_bf16(r.standard_normal((N, d)))
+    dO = lh.round_bf16(r.standard_normal((N, d)))
+    sz = lh.sizes(N, g["p"], g["L"], g["k"])
+    ctx = lh.head_forward(Q, K, V, sz, "bf16")
+    assert ctx["sel_idx"].tolist() == g["sel_idx"]
+    return g, sz, ctx, dO, lh.head_backward(ctx, dO, sz, "bf16")
+
+
+def test_backward_rounds_dOg_once_from_the_range_sums():
+    """dOg (the MMA operand dO~) is the exact sum of dO over R(l, i), rounded
+    once to bf16; the ranges are the hand-worked ones."""
+    g, sz, ctx, dO, b = _rounding_case()
+    exact = np.array([[math.fsum(dO[lo:hi + 1, c]) for c in range(dO.shape[1])]
+                      for lo, hi in g["scatter_bwd_ranges"]])
+    assert np.array_equal(b["dOg"], lh.round_bf16(exact))
+    assert not np.array_equal(lh.round_bf16(exact), exact)  # the rounding matters here
+
+
+def test_backward_forms_D_from_the_stored_operands():
+    """D_j = sum_c dOg_jc Og_jc with both factors as stored (bf16), not from the
+    unrounded range sums."""
+    g, sz, ctx, dO, b = _rounding_case()
+    assert np.array_equal(ctx["Og"], lh.round_bf16(ctx["Og"]))
+    D = [math.fsum(b["dOg"][j] * ctx["Og"][j]) for j in range(sz.S)]
+    assert np.allclose(b["D"], D, rtol=1e-15, atol=1e-15)
+    exact = np.array([[math.fsum(dO[lo:hi + 1, c]) for c in range(dO.shape[1])]
+                      for lo, hi in g["scatter_bwd_ranges"]])
+    D_unrounded = [math.fsum(exact[j] * ctx["Og"][j]) for j in range(sz.S)]
+    assert np.max(np.abs(np.array(D_unrounded) - b["D"])) > 1e-6
+
+
+def test_backward_rounds_gathered_gradients_before_the_pool_backward():
+    """dQg, dKg, dVg are stored in bf16 and the per-token gradient sums the
+    stored values with the hand-worked weights 1/p^l, rounding once at the
+    end; summing the unrounded values first gives different bits."""
+    g, sz, ctx, dO, b = _rounding_case()
+    exact = lh.causal_attention_bwd(ctx["Qg"], ctx["Kg"], ctx["Vg"], b["dOg"], ctx["lse"], b["D"])
+    differs = False
+    for key, full in zip(("dQ", "dK", "dV"), exact):
+        stored = b[key + "g"]
+        assert np.array_equal(stored, lh.round_bf16(full))
+        want = np.zeros_like(b[key])
+        alt = np.zeros_like(b[key])
+        for t, terms in enumerate(g["gather_bwd_terms"]):
+            for c in range(stored.shape[1]):
+                want[t, c] = math.fsum(w * stored[j, c] for j, w in terms)
+                alt[t, c] = math.fsum(w * full[j, c] for j, w in terms)
+        assert np.array_equal(b[key], lh.round_bf16(want))
+        differs |= not np.array_equal(lh.round_bf16(alt), b[key])
+    assert differs, "the case does not tell the two rounding orders apart"
+
+
 def test_planted_mistakes_are_caught():
     """A transposed operand or a dropped term in the oracle fails a pin."""
     p, L, N, k, d = 2, 3, 16, 1, 4
