@@ -19,7 +19,7 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
                                void* dK, void* dV, float* dq_acc, cudaStream_t st);
 cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                   const float* lse, const void* dO, const float* D, void* dQ,
-                                  void* dK, void* dV, cudaStream_t st);
+                                  void* dK, void* dV, float* dq_acc, cudaStream_t st);
 
 namespace {
 std::atomic<int> g_deterministic{0};
@@ -29,11 +29,11 @@ int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 void set_deterministic(int on) { g_deterministic.store(on != 0); }
 int deterministic() { return g_deterministic.load(); }
 
-// [D when the caller passes none | bf16, d = 64: fp32 dQ accumulator of the
-// fused schedule, BH * S * 64 floats]
+// [D when the caller passes none | bf16: fp32 dQ accumulator of the fused
+// schedule, BH * S * d floats]
 int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int d, int dtype) {
   const int64_t d_bytes = align256(BH * S * 4);
-  return dtype == LH_BF16 && d == kD ? d_bytes + align256(BH * S * kD * 4) : d_bytes;
+  return dtype == LH_BF16 ? d_bytes + align256(BH * S * d * 4) : d_bytes;
 }
 
 cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, int dtype, const void* Qg, const void* Kg,
@@ -58,14 +58,13 @@ cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, int dtype, const void*
   if (dtype == LH_F32)
     return launch_attn_bwd_f32(BH, S, d, (const float*)Qg, (const float*)Kg, (const float*)Vg, lse,
                                (const float*)dOg, D, (float*)dQg, (float*)dKg, (float*)dVg, st);
-  // d = 128: the two-kernel schedule (no fp32 dQ accumulator)
-  if (d == 128)
-    return launch_attn_bwd_tc128(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, st);
   // Without a workspace (the allocation-free entry point) or in deterministic
   // mode the two-kernel schedule runs; otherwise the fused one.
   float* dq_acc = (ws != nullptr && !deterministic())
                       ? reinterpret_cast<float*>(static_cast<char*>(ws) + align256(BH * S * 4))
                       : nullptr;
+  if (d == 128)
+    return launch_attn_bwd_tc128(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, dq_acc, st);
   return launch_attn_bwd_tc(BH, S, Qg, Kg, Vg, lse, dOg, D, dQg, dKg, dVg, dq_acc, st);
 }
 

@@ -4,17 +4,25 @@
 // "梯度流").  With P = exp(s - lse), dP = dO V^T, dS = P (dP - D),
 // D = rowsum(dO O):  dV = P^T dO,  dK = dS^T Q / sqrt(d),  dQ = dS K / sqrt(d).
 //
-// Two kernels, no atomics (the d = 64 library's deterministic schedule):
-//  - dk/dv: a CTA per 128-key tile streams 64-query chunks from its
-//    diagonal on.  TMEM: S^T [0,64) and dP^T [64,128) (lane = key), dV
-//    [128,256), dK [256,384), and P^T as bf16 pairs [384,416), the TMEM A
-//    operand of dV += P^T dO.  dS^T goes to swizzled K-major shared memory,
-//    the A operand of dK += dS^T Q.  With d = 128 the two accumulators take
-//    256 columns, so a step streams 64 queries: S^T and dP^T are N = 64
-//    products, dV and dK N = 128 ones;
-//  - dq: a CTA per 128-query tile streams 64-key chunks up to its diagonal:
-//    S = Q K^T and dP = dO V^T (lane = query) in TMEM [0,64) and [64,128),
-//    dS to shared memory, dQ += dS K in TMEM [128,256).
+// dk/dv kernel: a CTA per 128-key tile streams 64-query chunks from its
+// diagonal on.  TMEM: S^T [0,64) and dP^T [64,128) (lane = key), dV
+// [128,256), dK [256,384), and P^T as bf16 pairs [448,480), the TMEM A
+// operand of dV += P^T dO.  dS^T goes to swizzled K-major shared memory,
+// the A operand of dK += dS^T Q.  With d = 128 the two accumulators take 256
+// columns, so a step streams 64 queries: S^T and dP^T are N = 64 products,
+// dV and dK N = 128 ones.  Two schedules:
+//  - fused (default): the same kernel also forms each chunk's dQ share, and
+//    forms it transposed, dQ^T = K^T dS^T (M = 128 channels, N = 64 queries:
+//    TMEM [384,448), lane = channel), with both operands read MN-major from
+//    the resident K tile and the dS^T tile.  The element-wise threads stage
+//    it into four 64-query x 32-channel fp32 boxes and the MMA thread
+//    reduce-adds them with TMA into an fp32 dQ accumulator (run-to-run
+//    order, so the last bits of dQ vary); a rounding kernel scales it into
+//    dQ.  P and dS are formed once;
+//  - deterministic: no dQ share; a dq kernel, one CTA per 128-query tile
+//    streaming 64-key chunks up to its diagonal: S = Q K^T and dP = dO V^T
+//    (lane = query) in TMEM [0,64) and [64,128), dS to shared memory,
+//    dQ += dS K in TMEM [128,256).
 // The element-wise threads copy their S/dP columns out of TMEM and release
 // them at once, so the next step's S and dP products run while they compute
 // P and dS.  lse (times log2 e) and D of the streamed queries are staged in
@@ -31,6 +39,8 @@
 namespace lh {
 
 bool make_tile_map_d(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows, int d);
+bool make_acc_map_d(CUtensorMap* map, const float* ptr, int64_t rows, int d, int box_rows);
+cudaError_t launch_dq_round(const float* acc, void* dQ, int64_t n, float scale, cudaStream_t st);
 
 namespace {
 
@@ -114,6 +124,18 @@ __device__ __forceinline__ void gemm_acc_ts(uint32_t d, uint32_t a_tmem, uint32_
     mma_bf16_ts(d, a_tmem + 8 * kk, desc_add(db, kk * 2048), idesc, (acc || kk > 0) ? 1u : 0u);
 }
 
+// D[tmem] = K^T (128 channels x 128 keys) * dS^T (128 keys x 64 queries): the
+// transposed dQ share.  A is the resident K tile read MN-major (its two
+// 64-channel halves are the two M atoms, kHalfR apart); B is the dS^T tile
+// read MN-major (one 64-query atom).  K = keys: 16 key rows = 2048 bytes.
+__device__ __forceinline__ void gemm_dqt(uint32_t d, uint32_t k_tile, uint32_t dst_tile) {
+  constexpr uint32_t idesc = idesc_bf16(kRows, kC, true, true);
+  const uint64_t da = sw128_desc(k_tile, kHalfR, 1024), db = sw128_desc(dst_tile, kWide, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kRows / 16; ++kk)
+    mma_bf16(d, desc_add(da, kk * 2048), desc_add(db, kk * 2048), idesc, kk > 0 ? 1u : 0u);
+}
+
 // Both 64-column halves of a box_rows-row tile, completing on one barrier.
 __device__ __forceinline__ void load_tile(uint32_t dst, uint32_t half, const CUtensorMap* map, int row,
                                           uint32_t bar) {
@@ -129,23 +151,44 @@ struct KV {
   static constexpr uint32_t kOffQ = 2 * kTileR;                   // kStages chunks
   static constexpr uint32_t kOffG = kOffQ + kStages * kTileC;     // dO, kStages chunks
   static constexpr uint32_t kOffDST = kOffG + kStages * kTileC;   // dS^T (128 keys x 64 queries)
-  static constexpr uint32_t kOffL = kOffDST + kWide;              // kStages x 64 lse * log2 e
+  static constexpr uint32_t kStageBox = kC * 32 * 4;              // 8 KB: 64 queries x 32 channels fp32
+  static constexpr uint32_t kOffStage = kOffDST + kWide;          // 4 dQ share boxes (fused)
+  static constexpr uint32_t kOffL = kOffStage + 4 * kStageBox;    // kStages x 64 lse * log2 e
   static constexpr uint32_t kOffDv = kOffL + kStages * kC * 4;    // kStages x 64 D
   static constexpr uint32_t kOffBar = kOffDv + kStages * kC * 4;
   static constexpr uint32_t kBarKV = 0, kBarFull = 8, kBarEmpty = kBarFull + 8 * kStages,
                             kBarSP = kBarEmpty + 8 * kStages, kBarPDS = kBarSP + 8,
                             kBarAcc = kBarPDS + 8, kBarDrain = kBarAcc + 8, kBarTF = kBarDrain + 8,
-                            kBarPF = kBarTF + 8, kSlotTmem = kBarPF + 8, kSlotAbort = kSlotTmem + 4;
+                            kBarPF = kBarTF + 8, kBarQD = kBarPF + 8, kBarBF = kBarQD + 8,
+                            kSlotTmem = kBarBF + 8, kSlotAbort = kSlotTmem + 4;
   static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-  static constexpr uint32_t kColDV = 2 * kC, kColDK = kColDV + kD128, kColPT = kColDK + kD128;
+  static constexpr uint32_t kColDV = 2 * kC, kColDK = kColDV + kD128, kColDQT = kColDK + kD128,
+                            kColPT = kColDQT + kC;
   static_assert(kColPT + kC / 2 <= 512, "TMEM columns");
   static_assert(kSlotAbort + 4 <= 256, "barrier area");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
+// This thread's channel (TMEM lane) of 32 queries of a dQ^T share into
+// the staging box of its 32-channel block: query q is row q of the box
+// (128 bytes, 128-byte swizzle: 16-byte chunk j of row q at j ^ (q % 8)).
+__device__ __forceinline__ void stage_dqt32(uint32_t taddr, uint32_t box, int q0, int ch) {
+  float v[32];
+  tmem_ld32(taddr, v);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int q = q0 + i;
+    const uint32_t addr = box + q * 128 + ((((ch >> 2) ^ (q & 7))) << 4) + (ch & 3) * 4;
+    asm volatile("st.shared.f32 [%0], %1;\n" ::"r"(addr), "f"(v[i]) : "memory");
+  }
+}
+
+template <bool kFused>
 __global__ void __maxnreg__(168)
 attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
+                           const __grid_constant__ CUtensorMap tmDQ,
                            const float* __restrict__ lse, const float* __restrict__ Dv,
                            bf16* __restrict__ dK, bf16* __restrict__ dV, int S, float sl2, float scale,
                            int tiles_on_y, unsigned int* __restrict__ status) {
@@ -176,7 +219,9 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
     mbar_init(bars + L::kBarAcc, 1);
     mbar_init(bars + L::kBarDrain, 1);
     mbar_init(bars + L::kBarTF, kEw);  // S^T/dP^T copied out of TMEM
-    mbar_init(bars + L::kBarPF, 1);    // P^T/dS^T consumed by the dV/dK products
+    mbar_init(bars + L::kBarPF, 1);    // P^T/dS^T consumed (and the dQ share complete)
+    mbar_init(bars + L::kBarQD, kEw);  // a dQ share read out of TMEM and staged
+    mbar_init(bars + L::kBarBF, 1);    // the staging boxes read by the last reduce
     *abort = 0;
     fence_mbar_init();
   }
@@ -236,6 +281,14 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
         tc_fence_after();
         issue_sp(0);
       }
+      // dQ share j: issued as step j's last MMA, staged by the element-wise
+      // warps after step j+1's P/dS hand-off (QD), reduced from here into
+      // rows [k0 + kC j, +kC) of the accumulator; its boxes are released
+      // (BF) one step later.
+      auto reduce_share = [&](int j) {
+        for (int b = 0; b < 4; ++b)
+          tma_reduce_add_2d(&tmDQ, 32 * b, row0 + k0 + j * kC, base + L::kOffStage + b * L::kStageBox);
+      };
       for (int t = 0; ok && t < nq; ++t) {
         const int s = t % kStages;
         // S^T/dP^T of step t copied out: start step t+1's while step t computes
@@ -246,14 +299,36 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
           if (!(ok = mbar_wait(bars + L::kBarFull + 8 * s1, u1 & 1, abort, status))) break;
           issue_sp(s1);
         }
+        if constexpr (kFused) {
+          if (t >= 2) {  // share t-2's reduce has read the boxes
+            bulk_wait_read();
+            mbar_arrive(bars + L::kBarBF);
+          }
+        }
         if (!(ok = mbar_wait(bars + L::kBarPDS, t & 1, abort, status))) break;
         tc_fence_after();
         gemm_acc_ts(tmem + L::kColDV, tmem + L::kColPT, base + L::kOffG + s * kTileC, t > 0);  // dV += P^T dO
         gemm_acc(tmem + L::kColDK, base + L::kOffDST, base + L::kOffQ + s * kTileC, t > 0);    // dK += dS^T Q
+        if constexpr (kFused) {
+          if (t >= 1) {  // share t-1 out of TMEM and staged
+            if (!(ok = mbar_wait(bars + L::kBarQD, (t - 1) & 1, abort, status))) break;
+            tc_fence_after();
+            reduce_share(t - 1);
+          }
+          gemm_dqt(tmem + L::kColDQT, base + L::kOffK, base + L::kOffDST);  // share t = K^T dS^T
+        }
         mma_commit(bars + L::kBarPF);
         mma_commit(bars + L::kBarEmpty + 8 * s);
       }
       if (ok) mma_commit(bars + L::kBarAcc);
+      if constexpr (kFused) {
+        if (ok && nq >= 2) {
+          bulk_wait_read();
+          mbar_arrive(bars + L::kBarBF);
+        }
+        if (ok && mbar_wait(bars + L::kBarQD, (nq - 1) & 1, abort, status)) reduce_share(nq - 1);
+        bulk_wait_all();  // the reduces are complete before the CTA exits
+      }
       mma_commit(bars + L::kBarDrain);
       wait_drain(bars + L::kBarDrain, 0);
     }
@@ -264,6 +339,16 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
     const int key = k0 + r;
     const int col0 = grp * 32;     // this group's 32 query columns of the step
     const uint32_t lane_base = tmem + ((uint32_t)(wr * 32) << 16);
+    // share j: wait until share j-1's reduce has read the boxes, stage this
+    // thread's channel (lane r) for the group's 32 queries, arrive
+    auto stage_share = [&](int j) -> bool {
+      if (j >= 1 && !mbar_wait(bars + L::kBarBF, (j - 1) & 1, abort, status)) return false;
+      stage_dqt32(lane_base + L::kColDQT + col0, base + L::kOffStage + wr * L::kStageBox, col0, lane);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bars + L::kBarQD);
+      return true;
+    };
     const float2 sc2 = make_float2(sl2, sl2);
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
@@ -312,10 +397,18 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + L::kBarPDS);
+      if constexpr (kFused) {
+        // share t-1 (complete: PF above) leaves TMEM while dV/dK of step t run
+        if (t >= 1) ok = stage_share(t - 1);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      }
     }
     if (ok) ok = mbar_wait(bars + L::kBarAcc, 0, abort, status);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
+      if constexpr (kFused) {
+        if (nq > 0) stage_share(nq - 1);
+      }
       // group 0 writes dV, group 1 dK: 128 columns each, 32 at a time
 #pragma unroll
       for (int piece = 0; piece < 4; ++piece) {
@@ -523,7 +616,7 @@ attn_bwd_dq_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
 
 cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                   const float* lse, const void* dO, const float* D, void* dQ,
-                                  void* dK, void* dV, cudaStream_t st) {
+                                  void* dK, void* dV, float* dq_acc, cudaStream_t st) {
   // Tiles that stay resident in a CTA have 128 rows; streamed chunks 64.
   CUtensorMap qR, gR, kR, vR, qC, gC, kC_, vC;
   const int64_t rows = BH * S;
@@ -535,8 +628,11 @@ cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
   unsigned int* status = device_status_ptr();
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc128_kernel,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc128_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, KV::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_tc128_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, KV::kSmemBytes);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(attn_bwd_dq_tc128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              QQ::kSmemBytes);
@@ -549,9 +645,22 @@ cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
   const int ty = ntiles <= 65535 ? 1 : 0;
   if (!ty && BH > 65535) return cudaErrorInvalidConfiguration;
   const dim3 grid = ty ? dim3((unsigned)BH, ntiles) : dim3(ntiles, (unsigned)BH);
-  attn_bwd_dkdv_tc128_kernel<<<grid, kThreads, KV::kSmemBytes, st>>>(
-      qC, kR, vR, gC, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2, scale, ty,
-      status);
+  if (dq_acc != nullptr) {
+    const int64_t n = rows * kD128;
+    CUtensorMap accM;
+    if (!make_acc_map_d(&accM, dq_acc, rows, kD128, kC)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, (size_t)n * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    attn_bwd_dkdv_tc128_kernel<true><<<grid, kThreads, KV::kSmemBytes, st>>>(
+        qC, kR, vR, gC, accM, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV), (int)S, sl2,
+        scale, ty, status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_dq_round(dq_acc, dQ, n, scale, st);
+  }
+  attn_bwd_dkdv_tc128_kernel<false><<<grid, kThreads, KV::kSmemBytes, st>>>(
+      qC, kR, vR, gC, qC /* no dQ shares */, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV),
+      (int)S, sl2, scale, ty, status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_bwd_dq_tc128_kernel<<<grid, kThreads, QQ::kSmemBytes, st>>>(
