@@ -148,13 +148,13 @@ class Layer:
             ck(L.lh_gather(pl, t["Q"], t["K"], t["V"], p["pQ"], p["pK"], p["pV"], p["sel"],
                            p["Qg"], p["Kg"], p["Vg"], st), name)
         elif name == "attn_fwd":
-            ck(L.lh_attn_fwd(BH, S, 64, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], st), name)
+            ck(L.lh_attn_fwd(BH, S, r.c.d, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], st), name)
         elif name == "scatter":
             ck(L.lh_scatter(pl, p["Og"], p["slot"], t["O"], st), name)
         elif name == "scatter_bwd":
             ck(L.lh_scatter_bwd(pl, t["dO"], p["Og"], p["sel"], p["dOg"], p["D"], st), name)
         elif name == "attn_bwd":
-            ck(L.lh_attn_bwd(BH, S, 64, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], p["dOg"],
+            ck(L.lh_attn_bwd(BH, S, r.c.d, code, p["Qg"], p["Kg"], p["Vg"], p["Og"], p["lse"], p["dOg"],
                              p["D"], p["dQg"], p["dKg"], p["dVg"], p["aws"], r.attn_bwd_ws_bytes, st), name)
         elif name == "gather_bwd":
             ck(L.lh_gather_bwd(pl, p["dQg"], p["dKg"], p["dVg"], p["slot"], t["dQ"], t["dK"], t["dV"], st), name)
@@ -288,8 +288,8 @@ def timed_steps(layer, st, steps, backward=True):
     return total / steps, [x / steps for x in per_stage]
 
 
-def dense_sdpa_ms(H, N, steps=3, backward=True):
-    q = torch.randn(1, H, N, 64, device="cuda", dtype=torch.bfloat16, requires_grad=backward)
+def dense_sdpa_ms(H, N, steps=3, backward=True, d=64):
+    q = torch.randn(1, H, N, d, device="cuda", dtype=torch.bfloat16, requires_grad=backward)
     k = torch.randn_like(q, requires_grad=backward)
     v = torch.randn_like(q, requires_grad=backward)
     g = torch.randn_like(q)
@@ -316,8 +316,8 @@ def workload_extras(w, fwd_ms, fb_ms, dense_steps=3):
            "fwd_mtok_s": w.B * w.N / (fwd_ms * 1e-3) / 1e6,
            "fwd_bwd_mtok_s": w.B * w.N / (fb_ms * 1e-3) / 1e6}
     try:
-        sd_f = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False)
-        sd_fb = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True)
+        sd_f = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False, d=w.d)
+        sd_fb = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True, d=w.d)
         out["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb,
                                    "speedup_fwd": sd_f / fwd_ms, "speedup_fwd_bwd": sd_fb / fb_ms}
     except Exception as e:  # comparator only

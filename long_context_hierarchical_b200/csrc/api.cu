@@ -72,7 +72,7 @@ Geo make_geo(const lh_plan& p) {
 
 static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
-int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype);
+int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int d, int dtype);
 
 }  // namespace lh
 
@@ -113,7 +113,7 @@ lh_status lh_plan_init(const lh_config* cfg, lh_plan* out) {
   }
   if (c.N % P[c.L - 1] != 0) return fail(LH_ERR_INVALID_ARG, "N must be a multiple of p^(L-1)");
   if (c.dtype != LH_F32 && c.dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
-  if (c.d != kD) return fail(LH_ERR_UNSUPPORTED, "only d = 64 is built");
+  if (c.d != 64 && c.d != 128) return fail(LH_ERR_UNSUPPORTED, "only d in {64, 128} is built");
   if (c.p != 2 && c.p != 4) return fail(LH_ERR_UNSUPPORTED, "only p in {2, 4} is built");
   if (c.L > 5) return fail(LH_ERR_UNSUPPORTED, "only L <= 5 is built");
   if (P[c.L - 1] > 256) return fail(LH_ERR_UNSUPPORTED, "only p^(L-1) <= 256 is built");
@@ -181,7 +181,7 @@ lh_status lh_plan_init(const lh_config* cfg, lh_plan* out) {
   p.ws_dQg = o; o = align256(o + BH * p.S * row);
   p.ws_dKg = o; o = align256(o + BH * p.S * row);
   p.ws_dVg = o; o = align256(o + BH * p.S * row);
-  p.attn_bwd_ws_bytes = attn_bwd_ws_bytes(BH, p.S, c.dtype);
+  p.attn_bwd_ws_bytes = attn_bwd_ws_bytes(BH, p.S, c.d, c.dtype);
   p.ws_attn = o; o = align256(o + p.attn_bwd_ws_bytes);
   const int64_t bwd = o;
   p.ws_bytes = fwd > bwd ? fwd : bwd;
@@ -282,7 +282,7 @@ static lh_status check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
   if (BH < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "BH and S must be >= 1");
   if (S >= (int64_t(1) << 31)) return fail(LH_ERR_INVALID_ARG, "S must stay below 2^31");
   if (dtype != LH_F32 && dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
-  if (d != kD) return fail(LH_ERR_UNSUPPORTED, "only d = 64 is built");
+  if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "only d in {64, 128} is built");
   if (dtype == LH_BF16 && BH > ((int64_t(1) << 31) - 1) / S)
     return fail(LH_ERR_UNSUPPORTED, "bf16 attention needs BH * S < 2^31 (TMA row coordinates)");
   return LH_OK;
@@ -293,7 +293,7 @@ lh_status lh_attn_fwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
   Range range("lh_attn_fwd");
   LH_TRY(check_attn(BH, S, d, dtype));
   LH_CHECK_PTR(Qg); LH_CHECK_PTR(Kg); LH_CHECK_PTR(Vg); LH_CHECK_PTR(Og); LH_CHECK_PTR(lse);
-  LH_TRY(cuda_status(launch_attn_fwd(BH, S, dtype, Qg, Kg, Vg, Og, lse, as_cuda(stream)),
+  LH_TRY(cuda_status(launch_attn_fwd(BH, S, d, dtype, Qg, Kg, Vg, Og, lse, as_cuda(stream)),
                      "lh_attn_fwd"));
   return ok();
 }
@@ -302,7 +302,7 @@ void lh_set_deterministic(int on) { set_deterministic(on); }
 
 int64_t lh_attn_bwd_ws_bytes(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
   if (check_attn(BH, S, d, dtype) != LH_OK) return -1;
-  return attn_bwd_ws_bytes(BH, S, dtype);
+  return attn_bwd_ws_bytes(BH, S, d, dtype);
 }
 
 lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
@@ -315,13 +315,13 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
   LH_CHECK_PTR(dQg); LH_CHECK_PTR(dKg); LH_CHECK_PTR(dVg);
   if (D == nullptr) LH_CHECK_PTR(Og);
   else LH_CHECK_PTR(D);
-  const int64_t need = attn_bwd_ws_bytes(BH, S, dtype);
+  const int64_t need = attn_bwd_ws_bytes(BH, S, d, dtype);
   if (need > 0) {
     LH_CHECK_PTR(ws);
     if ((int64_t)ws_bytes < need)
       return fail(LH_ERR_WORKSPACE, "lh_attn_bwd workspace smaller than lh_attn_bwd_ws_bytes()");
   }
-  LH_TRY(cuda_status(launch_attn_bwd(BH, S, dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg, dKg, dVg, ws,
+  LH_TRY(cuda_status(launch_attn_bwd(BH, S, d, dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg, dKg, dVg, ws,
                                      as_cuda(stream)), "lh_attn_bwd"));
   return ok();
 }
@@ -395,7 +395,7 @@ lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const vo
   }
   {
     Range r("attn_fwd");
-    LH_TRY(cuda_status(launch_attn_fwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, st),
+    LH_TRY(cuda_status(launch_attn_fwd(BH, plan->S, plan->c.d, plan->c.dtype, Qg, Kg, Vg, Og, lse, st),
                        "lh_forward/attention"));
   }
   {
@@ -435,7 +435,7 @@ lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void
   }
   {
     Range r("attn_bwd");
-    LH_TRY(cuda_status(launch_attn_bwd(BH, plan->S, plan->c.dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg,
+    LH_TRY(cuda_status(launch_attn_bwd(BH, plan->S, plan->c.d, plan->c.dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg,
                                        dKg, dVg, aws, st), "lh_backward/attention"));
   }
   {

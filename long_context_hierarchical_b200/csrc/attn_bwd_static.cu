@@ -8,7 +8,7 @@
 
 namespace lh {
 
-cudaError_t launch_rowdot(int64_t rows, int dtype, const void* dO, const void* O, float* D,
+cudaError_t launch_rowdot(int64_t rows, int d, int dtype, const void* dO, const void* O, float* D,
                           cudaStream_t st);
 
 namespace {
@@ -53,7 +53,7 @@ extern "C" lh_status lh_attn_bwd_static(int64_t BH, int64_t S, int32_t d, int32_
   if (BH < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "BH and S must be >= 1");
   if (dtype != LH_F32 && dtype != LH_BF16)
     return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
-  if (d != kD) return fail(LH_ERR_UNSUPPORTED, "only d = 64 is built");
+  if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "only d in {64, 128} is built");
   if (BH > kStaticRows / S)
     return fail(LH_ERR_WORKSPACE,
                 "lh_attn_bwd_static: BH * S exceeds LH_ATTN_BWD_STATIC_MAX_ROWS (1048576 rows)");
@@ -64,9 +64,9 @@ extern "C" lh_status lh_attn_bwd_static(int64_t BH, int64_t S, int32_t d, int32_
   lh_status s = cuda_status(scratch_on_current_device(&D), "lh_attn_bwd_static/scratch");
   if (s != LH_OK) return s;
   cudaStream_t st = as_cuda(stream);
-  s = cuda_status(launch_rowdot(BH * S, dtype, dOg, Og, D, st), "lh_attn_bwd_static/rowdot");
+  s = cuda_status(launch_rowdot(BH * S, d, dtype, dOg, Og, D, st), "lh_attn_bwd_static/rowdot");
   if (s != LH_OK) return s;
-  s = cuda_status(launch_attn_bwd(BH, S, dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg, dKg, dVg,
+  s = cuda_status(launch_attn_bwd(BH, S, d, dtype, Qg, Kg, Vg, Og, lse, dOg, D, dQg, dKg, dVg,
                                   nullptr, st),
                   "lh_attn_bwd_static");
   if (s != LH_OK) return s;

@@ -689,6 +689,15 @@ constexpr int kStep = 128;  // streamed rows per step (64 measured slower: N=64 
 
 }  // namespace
 
+// dQ = scale * acc, n elements (a multiple of 8), rounded to bf16.
+cudaError_t launch_dq_round(const float* acc, void* dQ, int64_t n, float scale, cudaStream_t st) {
+  const int64_t n8 = n / 8;
+  const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
+  dq_round_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(acc), static_cast<uint4*>(dQ),
+                                          n8, scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void* K, const void* V,
                                const float* lse, const void* dO, const float* D, void* dQ,
                                void* dK, void* dV, float* dq_acc, cudaStream_t st) {
@@ -734,11 +743,7 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
         0.125f, ty, status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int64_t n8 = n / 8;
-    const int blocks = (int)std::min<int64_t>((n8 + 255) / 256, 148 * 8);
-    dq_round_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
-                                            static_cast<uint4*>(dQ), n8, 0.125f);
-    return cudaGetLastError();
+    return launch_dq_round(dq_acc, dQ, n, 0.125f, st);
   }
   attn_bwd_dkdv_tc_kernel<C, false><<<grid, F::kThreads, KV<C>::kSmemBytes, st>>>(
       qC, kR, vR, gC, qC /* no dQ shares */, lse, D, static_cast<bf16*>(dK), static_cast<bf16*>(dV),

@@ -321,6 +321,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
+// [rows, d] bf16 row-major (d a multiple of 64), boxes of box_rows rows x 64
+// columns, 128-byte swizzle: a row of d columns is d / 64 boxes side by side.
+bool make_tile_map_d(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [rows, 64] bf16 row-major, tiles of box_rows rows x 64 columns, 128-byte
 // swizzle.
 bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows) {
@@ -333,6 +347,21 @@ bool make_tile_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, d] fp32 row-major, boxes of box_rows rows x 32 columns (128 bytes),
+// 128-byte swizzle: the d = 128 dQ accumulator as the target of TMA
+// reduce-adds.
+bool make_acc_map_d(CUtensorMap* map, const float* ptr, int64_t rows, int d, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // [rows, 64] fp32 row-major, boxes of 128 rows x 16 columns (64 bytes),

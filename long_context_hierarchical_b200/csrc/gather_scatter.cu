@@ -10,9 +10,10 @@
 // Backward ("梯度流": dL -> scatter -> attention -> gather): the adjoints of
 // those two maps, plus the softmax-backward row term D.
 //
-// The gather and scatter-backward kernels give each row to 8 lanes: lane c
-// moves channels [8c, 8c+8) with 16-byte accesses, so a warp touches 4 whole
-// rows per instruction (the scatter and gather-backward split is below).  The scatter and gather-backward kernels are
+// Every kernel is a template on the head dimension D (64 or 128).  The gather
+// kernel gives each row to 8 lanes: lane c moves channels [8c, 8c+8) of each
+// 64-channel group with 16-byte accesses, so a warp touches 4 whole rows per
+// instruction (the split of the other kernels is below).  The scatter and gather-backward kernels are
 // token-centric and sum in a fixed (ascending-level) order: no atomics, and
 // the result does not depend on scheduling.
 #include "host.h"
@@ -32,7 +33,7 @@ __device__ __forceinline__ void copy_chunk(T* dst, const T* src) {
   for (int i = 0; i < (int)(8 * sizeof(T) / 16); ++i) d[i] = __ldg(s + i);
 }
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 gather_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
               const T* __restrict__ pQ, const T* __restrict__ pK, const T* __restrict__ pV,
@@ -43,12 +44,15 @@ gather_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K, const T* 
   if (row >= g.BH * g.S) return;
   const int64_t bh = row / g.S;
   const int64_t f = sel_idx[row];
-  const int64_t dst = row * kD + c * 8;
+  const int64_t dst = row * D + c * 8;
   if (f < 0 || f >= g.Ntot) {  // not a pyramid index: write zeros, read nothing
     const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    Vec8<T>::store(Qg + dst, z);
-    Vec8<T>::store(Kg + dst, z);
-    Vec8<T>::store(Vg + dst, z);
+#pragma unroll
+    for (int h = 0; h < D / 64; ++h) {
+      Vec8<T>::store(Qg + dst + 64 * h, z);
+      Vec8<T>::store(Kg + dst + 64 * h, z);
+      Vec8<T>::store(Vg + dst + 64 * h, z);
+    }
     return;
   }
   const int l = level_of(g, f);
@@ -56,15 +60,18 @@ gather_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K, const T* 
   int64_t src;
   const T *sq, *sk, *sv;
   if (l == 0) {
-    src = (bh * g.N + i) * kD;
+    src = (bh * g.N + i) * D;
     sq = Q; sk = K; sv = V;
   } else {
-    src = (bh * g.Npyr + g.pyr_off[l] + i) * kD;
+    src = (bh * g.Npyr + g.pyr_off[l] + i) * D;
     sq = pQ; sk = pK; sv = pV;
   }
-  copy_chunk(Qg + dst, sq + src + c * 8);
-  copy_chunk(Kg + dst, sk + src + c * 8);
-  copy_chunk(Vg + dst, sv + src + c * 8);
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
+    copy_chunk(Qg + dst + 64 * h, sq + src + c * 8 + 64 * h);
+    copy_chunk(Kg + dst + 64 * h, sk + src + c * 8 + 64 * h);
+    copy_chunk(Vg + dst + 64 * h, sv + src + c * 8 + 64 * h);
+  }
 }
 
 template <typename T>
@@ -93,10 +100,11 @@ __device__ __forceinline__ void store_stream<float>(float* p, const float (&x)[8
 // instruction-bound with 8 lanes per row) while every store instruction
 // still covers whole 32-byte sectors.
 constexpr int kLanesPerRow = 4;
-constexpr int kChunks = 8 / kLanesPerRow;  // 8-element chunks per lane
+template <int D>
+constexpr int kChunks = D / 8 / kLanesPerRow;  // 8-element chunks per lane
 constexpr int kRowsPerBlock4 = kThreads / kLanesPerRow;
 
-template <typename T, int LOGP, int L>
+template <typename T, int D, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
@@ -105,7 +113,7 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
-  const T* og = Og + bh * g.S * kD + c * 8;
+  const T* og = Og + bh * g.S * D + c * 8;
   const int S = (int)g.S;
   int32_t slot[L];
 #pragma unroll
@@ -113,17 +121,17 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
     const int i = ((t + 1) >> (LOGP * l)) - 1;
     slot[l] = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
   }
-  float a[kChunks][8];
+  float a[kChunks<D>][8];
 #pragma unroll
-  for (int k = 0; k < kChunks; ++k)
+  for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
   for (int l = 0; l < L; ++l) {  // ascending level
     if ((unsigned)slot[l] < (unsigned)S) {
-      const T* src = og + (int64_t)slot[l] * kD;
+      const T* src = og + (int64_t)slot[l] * D;
 #pragma unroll
-      for (int k = 0; k < kChunks; ++k) {
+      for (int k = 0; k < kChunks<D>; ++k) {
         float x[8];
         Vec8<T>::load(src + 8 * kLanesPerRow * k, x);
 #pragma unroll
@@ -131,19 +139,20 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
       }
     }
   }
-  T* dst = O + (bh * g.N + t) * kD + c * 8;
+  T* dst = O + (bh * g.N + t) * D + c * 8;
 #pragma unroll
-  for (int k = 0; k < kChunks; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
+  for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
 }
 
 constexpr int kBwdLanes = 4;  // lanes per slot row in the scatter backward (8 and 2 measured slower)
-constexpr int kBwdChunks = 8 / kBwdLanes;
+template <int D>
+constexpr int kBwdChunks = D / 8 / kBwdLanes;
 constexpr int kRowsPerBlockB = kThreads / kBwdLanes;
 
-template <typename T, int LOGP, int L>
+template <typename T, int D, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
-                   const int32_t* __restrict__ sel_idx, T* __restrict__ dOg, float* __restrict__ D) {
+                   const int32_t* __restrict__ sel_idx, T* __restrict__ dOg, float* __restrict__ Drow) {
   const int j = blockIdx.x * kRowsPerBlockB + (int)(threadIdx.x / kBwdLanes);
   const int c = threadIdx.x % kBwdLanes;
   const int S = (int)g.S, N = (int)g.N;
@@ -160,40 +169,40 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   const int sh = LOGP * l;
   const int lo = ((i + 1) << sh) - 1;
   const int hi = min(lo + (1 << sh) - 1, N - 1);
-  const T* src = dO + bh * g.N * kD + c * 8;
-  float acc[kBwdChunks][8];
+  const T* src = dO + bh * g.N * D + c * 8;
+  float acc[kBwdChunks<D>][8];
 #pragma unroll
-  for (int k = 0; k < kBwdChunks; ++k)
+  for (int k = 0; k < kBwdChunks<D>; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
   int t = lo;
   for (; t + 3 <= hi; t += 4) {  // four independent row loads in flight
 #pragma unroll
-    for (int k = 0; k < kBwdChunks; ++k) {
+    for (int k = 0; k < kBwdChunks<D>; ++k) {
       float x0[8], x1[8], x2[8], x3[8];
       const T* p = src + 8 * kBwdLanes * k;
-      Vec8<T>::load(p + (int64_t)t * kD, x0);
-      Vec8<T>::load(p + (int64_t)(t + 1) * kD, x1);
-      Vec8<T>::load(p + (int64_t)(t + 2) * kD, x2);
-      Vec8<T>::load(p + (int64_t)(t + 3) * kD, x3);
+      Vec8<T>::load(p + (int64_t)t * D, x0);
+      Vec8<T>::load(p + (int64_t)(t + 1) * D, x1);
+      Vec8<T>::load(p + (int64_t)(t + 2) * D, x2);
+      Vec8<T>::load(p + (int64_t)(t + 3) * D, x3);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[k][e] += ((x0[e] + x1[e]) + (x2[e] + x3[e]));
     }
   }
   for (; t <= hi; ++t) {
 #pragma unroll
-    for (int k = 0; k < kBwdChunks; ++k) {
+    for (int k = 0; k < kBwdChunks<D>; ++k) {
       float x[8];
-      Vec8<T>::load(src + 8 * kBwdLanes * k + (int64_t)t * kD, x);
+      Vec8<T>::load(src + 8 * kBwdLanes * k + (int64_t)t * D, x);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[k][e] += x[e];
     }
   }
   float dsum = 0.f;
 #pragma unroll
-  for (int k = 0; k < kBwdChunks; ++k) {
+  for (int k = 0; k < kBwdChunks<D>; ++k) {
     float o[8];
-    Vec8<T>::load(Og + r * kD + c * 8 + 8 * kBwdLanes * k, o);
+    Vec8<T>::load(Og + r * D + c * 8 + 8 * kBwdLanes * k, o);
 #pragma unroll
     for (int e = 0; e < 8; ++e) dsum = fmaf(Vec8<T>::rounded(acc[k][e]), o[e], dsum);
   }
@@ -201,11 +210,11 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   for (int m = 1; m < kBwdLanes; m <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, m);
   if (!live) return;
 #pragma unroll
-  for (int k = 0; k < kBwdChunks; ++k) Vec8<T>::store(dOg + r * kD + c * 8 + 8 * kBwdLanes * k, acc[k]);
-  if (c == 0) D[r] = dsum;
+  for (int k = 0; k < kBwdChunks<D>; ++k) Vec8<T>::store(dOg + r * D + c * 8 + 8 * kBwdLanes * k, acc[k]);
+  if (c == 0) Drow[r] = dsum;
 }
 
-template <typename T, int LOGP, int L>
+template <typename T, int D, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
@@ -215,28 +224,28 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   if (t >= (int)g.N) return;
   const int64_t bh = blockIdx.y;
   const int32_t* inv = slot_of + bh * g.Ntot;
-  const int64_t base = bh * g.S * kD + c * 8;
+  const int64_t base = bh * g.S * D + c * 8;
   const int S = (int)g.S;
   int32_t slot[L];
 #pragma unroll
   for (int l = 0; l < L; ++l) slot[l] = __ldg(inv + (int)g.flat_off[l] + (t >> (LOGP * l)));
-  const int64_t out = (bh * g.N + t) * kD + c * 8;
+  const int64_t out = (bh * g.N + t) * D + c * 8;
   const T* src[3] = {dQg, dKg, dVg};
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
-    float a[kChunks][8];
+    float a[kChunks<D>][8];
 #pragma unroll
-    for (int k = 0; k < kChunks; ++k)
+    for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
       for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
     for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
       if ((unsigned)slot[l] < (unsigned)S) {
-        const T* p = src[w] + base + (int64_t)slot[l] * kD;
+        const T* p = src[w] + base + (int64_t)slot[l] * D;
         const float wgt = 1.f / (float)(1 << (LOGP * l));
 #pragma unroll
-        for (int k = 0; k < kChunks; ++k) {
+        for (int k = 0; k < kChunks<D>; ++k) {
           float x[8];
           Vec8<T>::load(p + 8 * kLanesPerRow * k, x);
 #pragma unroll
@@ -245,7 +254,7 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
       }
     }
 #pragma unroll
-    for (int k = 0; k < kChunks; ++k) store_stream<T>(dst[w] + out + 8 * kLanesPerRow * k, a[k]);
+    for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst[w] + out + 8 * kLanesPerRow * k, a[k]);
   }
 }
 
@@ -259,17 +268,11 @@ cudaError_t launch_gather(const lh_plan& plan, const void* Q, const void* K, con
                           const int32_t* sel_idx, void* Qg, void* Kg, void* Vg, cudaStream_t st) {
   const Geo g = make_geo(plan);
   const unsigned b = blocks_for(g.BH * g.S);
-  if (plan.c.dtype == LH_BF16) {
-    using T = __nv_bfloat16;
-    gather_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)Q, (const T*)K, (const T*)V,
-                                             (const T*)pyrQ, (const T*)pyrK, (const T*)pyrV,
-                                             sel_idx, (T*)Qg, (T*)Kg, (T*)Vg);
-  } else {
-    using T = float;
-    gather_kernel<T><<<b, kThreads, 0, st>>>(g, (const T*)Q, (const T*)K, (const T*)V,
-                                             (const T*)pyrQ, (const T*)pyrK, (const T*)pyrV,
-                                             sel_idx, (T*)Qg, (T*)Kg, (T*)Vg);
-  }
+  with_type_dim(plan, [&]<typename T, int D>() {
+    gather_kernel<T, D><<<b, kThreads, 0, st>>>(g, (const T*)Q, (const T*)K, (const T*)V,
+                                                (const T*)pyrQ, (const T*)pyrK, (const T*)pyrV,
+                                                sel_idx, (T*)Qg, (T*)Kg, (T*)Vg);
+  });
   return cudaGetLastError();
 }
 
@@ -295,46 +298,46 @@ void with_levels(const Geo& g, F&& f) {
   }
 }
 
-template <typename T>
+template <typename T, int D>
 void scatter_t(const Geo& g, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
   const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
-    scatter_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+    scatter_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
   });
 }
 
 cudaError_t launch_scatter(const lh_plan& plan, const void* Og, const int32_t* slot_of, void* O,
                            cudaStream_t st) {
   const Geo g = make_geo(plan);
-  if (plan.c.dtype == LH_BF16) scatter_t<__nv_bfloat16>(g, Og, slot_of, O, st);
-  else scatter_t<float>(g, Og, slot_of, O, st);
+  with_type_dim(plan, [&]<typename T, int D>() { scatter_t<T, D>(g, Og, slot_of, O, st); });
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int D>
 void scatter_bwd_t(const Geo& g, const void* dO, const void* Og, const int32_t* sel_idx, void* dOg,
-                   float* D, cudaStream_t st) {
+                   float* Drow, cudaStream_t st) {
   const dim3 grid((unsigned)((g.S + kRowsPerBlockB - 1) / kRowsPerBlockB), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
-    scatter_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og, sel_idx,
-                                                              (T*)dOg, D);
+    scatter_bwd_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og,
+                                                                 sel_idx, (T*)dOg, Drow);
   });
 }
 
 cudaError_t launch_scatter_bwd(const lh_plan& plan, const void* dO, const void* Og,
-                               const int32_t* sel_idx, void* dOg, float* D, cudaStream_t st) {
+                               const int32_t* sel_idx, void* dOg, float* Drow, cudaStream_t st) {
   const Geo g = make_geo(plan);
-  if (plan.c.dtype == LH_BF16) scatter_bwd_t<__nv_bfloat16>(g, dO, Og, sel_idx, dOg, D, st);
-  else scatter_bwd_t<float>(g, dO, Og, sel_idx, dOg, D, st);
+  with_type_dim(plan, [&]<typename T, int D>() {
+    scatter_bwd_t<T, D>(g, dO, Og, sel_idx, dOg, Drow, st);
+  });
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int D>
 void gather_bwd_t(const Geo& g, const void* dQg, const void* dKg, const void* dVg,
                   const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
   const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
   with_levels(g, [&]<int LOGP, int L>() {
-    gather_bwd_kernel<T, LOGP, L><<<grid, kThreads, 0, st>>>(
+    gather_bwd_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(
         g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
   });
 }
@@ -343,8 +346,9 @@ cudaError_t launch_gather_bwd(const lh_plan& plan, const void* dQg, const void* 
                               const void* dVg, const int32_t* slot_of, void* dQ, void* dK,
                               void* dV, cudaStream_t st) {
   const Geo g = make_geo(plan);
-  if (plan.c.dtype == LH_BF16) gather_bwd_t<__nv_bfloat16>(g, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
-  else gather_bwd_t<float>(g, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
+  with_type_dim(plan, [&]<typename T, int D>() {
+    gather_bwd_t<T, D>(g, dQg, dKg, dVg, slot_of, dQ, dK, dV, st);
+  });
   return cudaGetLastError();
 }
 

@@ -18,6 +18,20 @@ lh_status ok();
 lh_status cuda_status(cudaError_t e, const char* where);
 
 Geo make_geo(const lh_plan& p);
+
+// Calls f.template operator()<T, D>() for the plan's storage type and head
+// dimension (d in {64, 128}, validated by lh_plan_init).
+template <typename F>
+void with_type_dim(const lh_plan& plan, F&& f) {
+  const bool bf = plan.c.dtype == LH_BF16;
+  if (plan.c.d == 128) {
+    if (bf) f.template operator()<__nv_bfloat16, 128>();
+    else f.template operator()<float, 128>();
+  } else {
+    if (bf) f.template operator()<__nv_bfloat16, 64>();
+    else f.template operator()<float, 64>();
+  }
+}
 // Device address of the status word that bounded waits set on timeout.
 unsigned int* device_status_ptr();
 bool aligned16(const void* ptr);
@@ -40,15 +54,18 @@ cudaError_t launch_scatter_bwd(const lh_plan& plan, const void* dO, const void* 
 cudaError_t launch_gather_bwd(const lh_plan& plan, const void* dQg, const void* dKg,
                               const void* dVg, const int32_t* slot_of, void* dQ, void* dK,
                               void* dV, cudaStream_t st);
-cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
+cudaError_t launch_attn_fwd(int64_t BH, int64_t S, int d, int dtype, const void* Qg, const void* Kg,
                             const void* Vg, void* Og, float* lse, cudaStream_t st);
-int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int dtype);
+int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int d, int dtype);
 void set_deterministic(int on);
 int deterministic();
-cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int dtype, const void* Qg, const void* Kg,
+cudaError_t launch_attn_bwd(int64_t BH, int64_t S, int d, int dtype, const void* Qg, const void* Kg,
                             const void* Vg, const void* Og, const float* lse, const void* dOg,
                             const float* D, void* dQg, void* dKg, void* dVg, void* ws,
                             cudaStream_t st);
+// bf16 attention with d = 128 (tcgen05).
+cudaError_t launch_attn_fwd_tc128(int64_t BH, int64_t S, const void* Q, const void* K,
+                                  const void* V, void* O, float* lse, cudaStream_t st);
 // One CTA waiting on a barrier nothing signals (the failure-path self-test).
 cudaError_t launch_wait_timeout_selftest(cudaStream_t st);
 

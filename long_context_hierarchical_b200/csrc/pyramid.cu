@@ -11,7 +11,8 @@
 // (batch, head), so every pyramid entry it writes lies inside its rows.  Per
 // step the warp covers 16 rows: lane = 8*rr + c holds column chunk c (8
 // channels, one 16-byte load for bf16) of the 4-row block rr, rows
-// [4 rr, 4 rr + 4).  Sums over 2 or 4 rows stay in the lane, sums over 8 and
+// [4 rr, 4 rr + 4), for each 64-channel group of the row in turn (one group
+// for d = 64, two for d = 128; the norm sums run over all groups).  Sums over 2 or 4 rows stay in the lane, sums over 8 and
 // 16 rows take one or two xor-shuffles across rr, and longer spans
 // accumulate across steps in registers.  Sums are fp32 and rounded once;
 // p^l is a power of two, so the mean's scaling is exact.  The norm sums run
@@ -65,7 +66,7 @@ __device__ __forceinline__ void store_mean(T* dst, const float (&s)[8], float in
   Vec8<T>::store(dst, m);
 }
 
-template <typename T, int LOGP, int L>
+template <typename T, int D, int LOGP, int L>
 __global__ void __launch_bounds__(128)
 pyramid_score_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K,
                      const T* __restrict__ V, T* __restrict__ pyrQ, T* __restrict__ pyrK,
@@ -82,121 +83,128 @@ pyramid_score_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K,
   const int64_t row0 = (gw % groups_per_head) * W;
   const int64_t N = g.N;
 
-  const T* src[3] = {Q + bh * N * kD, K + bh * N * kD, V ? V + bh * N * kD : nullptr};
-  T* dst[3] = {pyrQ ? pyrQ + bh * g.Npyr * kD : nullptr, pyrK ? pyrK + bh * g.Npyr * kD : nullptr,
-               pyrV ? pyrV + bh * g.Npyr * kD : nullptr};
+  constexpr int G = D / 64;  // 64-channel groups per row
+  const T* src[3] = {Q + bh * N * D, K + bh * N * D, V ? V + bh * N * D : nullptr};
+  T* dst[3] = {pyrQ ? pyrQ + bh * g.Npyr * D : nullptr, pyrK ? pyrK + bh * g.Npyr * D : nullptr,
+               pyrV ? pyrV + bh * g.Npyr * D : nullptr};
   float* sc = scores ? scores + bh * g.M : nullptr;
   const int ntens = pool ? 3 : 2;
 
   // Cross-step state: running sums of levels whose span exceeds 16 rows
   // (only p = 4, levels 3 and 4) and the running max of level 3's score.
-  float acc3[3][8], acc4[3][8];
+  float acc3[G][3][8], acc4[G][3][8];
   float runmax3 = -INFINITY;
 #pragma unroll
-  for (int t = 0; t < 3; ++t)
+  for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc3[t][e] = acc4[t][e] = 0.f;
+    for (int t = 0; t < 3; ++t)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc3[h][t][e] = acc4[h][t][e] = 0.f;
 
 #pragma unroll 1
   for (int s = 0; s < STEPS; ++s) {
     const int64_t blk = row0 + s * 16 + rr * 4;  // first row of this lane's block
-    Packed<T> raw[3][4];
-#pragma unroll
-    for (int t = 0; t < 3; ++t)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (t < ntens && blk + j < N) raw[t][j].load(src[t] + (blk + j) * kD + c * 8);
-        else raw[t][j].zero();
-      }
-
     double ssq[8];  // [0..3]: ||Q_row||^2 partials, [4..7]: ||K_row||^2 partials
 #pragma unroll
     for (int j = 0; j < 8; ++j) ssq[j] = 0.0;
 
 #pragma unroll
-    for (int t = 0; t < 3; ++t) {
-      if (t >= ntens) break;
-      float x[4][8];
+    for (int h = 0; h < G; ++h) {
+      const int col = c * 8 + 64 * h;  // first channel of this lane's chunk
+      Packed<T> raw[3][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) raw[t][j].unpack(x[j]);
-      if (score && t < 2) {
+      for (int t = 0; t < 3; ++t)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          double a = 0.0;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a = fma((double)x[j][e], (double)x[j][e], a);
-          ssq[t * 4 + j] = a;
+          if (t < ntens && blk + j < N) raw[t][j].load(src[t] + (blk + j) * D + col);
+          else raw[t][j].zero();
         }
-      }
-      if (!pool) continue;
-      // Level sums.  s2a/s2b: rows {0,1}/{2,3}; s4: the 4-row block.
-      float s2a[8], s2b[8], s4[8];
+
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        s2a[e] = x[0][e] + x[1][e];
-        s2b[e] = x[2][e] + x[3][e];
-        s4[e] = s2a[e] + s2b[e];
-      }
-      T* out = dst[t];
-      if (LOGP == 1) {
-        // p = 2: P = 2, 4, 8, 16 for levels 1..4.
-        if (L >= 2) {
-          const int64_t i = blk / 2;
-          if (blk < N) store_mean<T>(out + (g.pyr_off[1] + i) * kD + c * 8, s2a, 0.5f);
-          if (blk + 2 < N) store_mean<T>(out + (g.pyr_off[1] + i + 1) * kD + c * 8, s2b, 0.5f);
-        }
-        if (L >= 3 && blk < N) store_mean<T>(out + (g.pyr_off[2] + blk / 4) * kD + c * 8, s4, 0.25f);
-        if (L >= 4) {
-          float s8[8];
+      for (int t = 0; t < 3; ++t) {
+        if (t >= ntens) break;
+        float x[4][8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s8[e] = s4[e];
-          shfl_add8(s8, 8);
-          if ((rr & 1) == 0 && blk < N)
-            store_mean<T>(out + (g.pyr_off[3] + blk / 8) * kD + c * 8, s8, 0.125f);
-          if (L >= 5) {
-            shfl_add8(s8, 16);
-            if (rr == 0 && blk < N)
-              store_mean<T>(out + (g.pyr_off[4] + blk / 16) * kD + c * 8, s8, 0.0625f);
+        for (int j = 0; j < 4; ++j) raw[t][j].unpack(x[j]);
+        if (score && t < 2) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            double a = 0.0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a = fma((double)x[j][e], (double)x[j][e], a);
+            ssq[t * 4 + j] += a;
           }
         }
-      } else {
-        // p = 4: P = 4, 16, 64, 256 for levels 1..4.
-        if (L >= 2 && blk < N) store_mean<T>(out + (g.pyr_off[1] + blk / 4) * kD + c * 8, s4, 0.25f);
-        if (L >= 3) {
-          float s16[8];
+        if (!pool) continue;
+        // Level sums.  s2a/s2b: rows {0,1}/{2,3}; s4: the 4-row block.
+        float s2a[8], s2b[8], s4[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s16[e] = s4[e];
-          shfl_add8(s16, 8);
-          shfl_add8(s16, 16);
-          if (rr == 0 && blk < N)
-            store_mean<T>(out + (g.pyr_off[2] + blk / 16) * kD + c * 8, s16, 1.f / 16.f);
+        for (int e = 0; e < 8; ++e) {
+          s2a[e] = x[0][e] + x[1][e];
+          s2b[e] = x[2][e] + x[3][e];
+          s4[e] = s2a[e] + s2b[e];
+        }
+        T* out = dst[t];
+        if (LOGP == 1) {
+          // p = 2: P = 2, 4, 8, 16 for levels 1..4.
+          if (L >= 2) {
+            const int64_t i = blk / 2;
+            if (blk < N) store_mean<T>(out + (g.pyr_off[1] + i) * D + col, s2a, 0.5f);
+            if (blk + 2 < N) store_mean<T>(out + (g.pyr_off[1] + i + 1) * D + col, s2b, 0.5f);
+          }
+          if (L >= 3 && blk < N) store_mean<T>(out + (g.pyr_off[2] + blk / 4) * D + col, s4, 0.25f);
           if (L >= 4) {
+            float s8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc3[t][e] += s16[e];
-            if ((s & 3) == 3) {
-              if (rr == 0) {
-                const int64_t i = (row0 + s * 16) / 64;
-                store_mean<T>(out + (g.pyr_off[3] + i) * kD + c * 8, acc3[t], 1.f / 64.f);
-              }
-              if (L >= 5) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc4[t][e] += acc3[t][e];
-              }
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc3[t][e] = 0.f;
+            for (int e = 0; e < 8; ++e) s8[e] = s4[e];
+            shfl_add8(s8, 8);
+            if ((rr & 1) == 0 && blk < N)
+              store_mean<T>(out + (g.pyr_off[3] + blk / 8) * D + col, s8, 0.125f);
+            if (L >= 5) {
+              shfl_add8(s8, 16);
+              if (rr == 0 && blk < N)
+                store_mean<T>(out + (g.pyr_off[4] + blk / 16) * D + col, s8, 0.0625f);
             }
-            if (L >= 5 && (s & 15) == 15) {
-              if (rr == 0) {
-                const int64_t i = (row0 + s * 16) / 256;
-                store_mean<T>(out + (g.pyr_off[4] + i) * kD + c * 8, acc4[t], 1.f / 256.f);
-              }
+          }
+        } else {
+          // p = 4: P = 4, 16, 64, 256 for levels 1..4.
+          if (L >= 2 && blk < N) store_mean<T>(out + (g.pyr_off[1] + blk / 4) * D + col, s4, 0.25f);
+          if (L >= 3) {
+            float s16[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) acc4[t][e] = 0.f;
+            for (int e = 0; e < 8; ++e) s16[e] = s4[e];
+            shfl_add8(s16, 8);
+            shfl_add8(s16, 16);
+            if (rr == 0 && blk < N)
+              store_mean<T>(out + (g.pyr_off[2] + blk / 16) * D + col, s16, 1.f / 16.f);
+            if (L >= 4) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc3[h][t][e] += s16[e];
+              if ((s & 3) == 3) {
+                if (rr == 0) {
+                  const int64_t i = (row0 + s * 16) / 64;
+                  store_mean<T>(out + (g.pyr_off[3] + i) * D + col, acc3[h][t], 1.f / 64.f);
+                }
+                if (L >= 5) {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) acc4[h][t][e] += acc3[h][t][e];
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc3[h][t][e] = 0.f;
+              }
+              if (L >= 5 && (s & 15) == 15) {
+                if (rr == 0) {
+                  const int64_t i = (row0 + s * 16) / 256;
+                  store_mean<T>(out + (g.pyr_off[4] + i) * D + col, acc4[h][t], 1.f / 256.f);
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc4[h][t][e] = 0.f;
+              }
             }
           }
         }
       }
-    }
+    }  // 64-channel groups
 
     if (score) {
       // Reduce-scatter the 8 partials over the 8 column lanes: afterwards
@@ -249,7 +257,7 @@ pyramid_score_kernel(Geo g, const T* __restrict__ Q, const T* __restrict__ K,
   }
 }
 
-template <typename T, int LOGP, int L>
+template <typename T, int D, int LOGP, int L>
 cudaError_t launch_typed(const lh_plan& plan, const void* Q, const void* K, const void* V,
                          void* pyrQ, void* pyrK, void* pyrV, float* scores, bool pool,
                          bool score, cudaStream_t st) {
@@ -259,20 +267,20 @@ cudaError_t launch_typed(const lh_plan& plan, const void* Q, const void* K, cons
   const int64_t groups = (g.N + W - 1) / W;
   const int64_t warps = g.BH * groups;
   const int64_t blocks = (warps + 3) / 4;
-  pyramid_score_kernel<T, LOGP, L><<<(unsigned)blocks, 128, 0, st>>>(
+  pyramid_score_kernel<T, D, LOGP, L><<<(unsigned)blocks, 128, 0, st>>>(
       g, static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
       static_cast<T*>(pyrQ), static_cast<T*>(pyrK), static_cast<T*>(pyrV), scores, pool ? 1 : 0,
       score ? 1 : 0, groups);
   return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, int D>
 cudaError_t launch_levels(const lh_plan& plan, const void* Q, const void* K, const void* V,
                           void* pyrQ, void* pyrK, void* pyrV, float* scores, bool pool,
                           bool score, cudaStream_t st) {
   const int L = plan.c.L;
 #define LH_CASE(LOGP, LL)                                                                   \
-  if (L == LL) return launch_typed<T, LOGP, LL>(plan, Q, K, V, pyrQ, pyrK, pyrV, scores, pool, \
+  if (L == LL) return launch_typed<T, D, LOGP, LL>(plan, Q, K, V, pyrQ, pyrK, pyrV, scores, pool, \
                                                 score, st);
   if (plan.c.p == 2) {
     LH_CASE(1, 2) LH_CASE(1, 3) LH_CASE(1, 4) LH_CASE(1, 5)
@@ -289,11 +297,12 @@ cudaError_t launch_pyramid_score(const lh_plan& plan, const void* Q, const void*
                                  const void* V, void* pyrQ, void* pyrK, void* pyrV,
                                  float* scores, bool pool, bool score, cudaStream_t st) {
   if (plan.c.L < 2) return cudaSuccess;  // no coarse level and no candidates
-  if (plan.c.dtype == LH_BF16)
-    return launch_levels<__nv_bfloat16>(plan, Q, K, pool ? V : nullptr, pyrQ, pyrK, pyrV, scores,
-                                        pool, score, st);
-  return launch_levels<float>(plan, Q, K, pool ? V : nullptr, pyrQ, pyrK, pyrV, scores, pool,
-                              score, st);
+  cudaError_t e = cudaSuccess;
+  with_type_dim(plan, [&]<typename T, int D>() {
+    e = launch_levels<T, D>(plan, Q, K, pool ? V : nullptr, pyrQ, pyrK, pyrV, scores, pool, score,
+                            st);
+  });
+  return e;
 }
 
 }  // namespace lh

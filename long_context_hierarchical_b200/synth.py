@@ -50,6 +50,8 @@ WORKLOADS = {
     # the same budget chosen by hierarchical descent (k best per level, their children kept)
     "98k_descent_k1536": Workload("98k_descent_k1536", 1, 16, 98304, 64, "bf16", 4, 3, 1536, True,
                                   "descent"),
+    # head dimension 128 at the same bytes per token (8 heads x 128 channels)
+    "98k_d128_k1536": Workload("98k_d128_k1536", 1, 8, 98304, 128, "bf16", 4, 3, 1536, True),
 }
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -55,7 +55,8 @@ def test_plan_sizes_match_oracle(name):
     ((1, 2, 1024, 64, 4, 0, 1, "bf16"), lh.LH_ERR_INVALID_ARG),    # L < 1
     ((0, 2, 1024, 64, 4, 3, 1, "bf16"), lh.LH_ERR_INVALID_ARG),    # B < 1
     ((1, 2, 1024, 64, 4, 3, -1, "bf16"), lh.LH_ERR_INVALID_ARG),   # k < 0
-    ((1, 2, 1024, 128, 4, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),   # d = 128
+    ((1, 2, 1024, 96, 4, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # d = 96
+    ((1, 2, 1024, 128, 4, 3, 1, "bf16"), None),                    # d = 128: built
     ((1, 2, 1152, 64, 3, 3, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # p = 3
     ((1, 2, 4096, 64, 2, 6, 1, "bf16"), lh.LH_ERR_UNSUPPORTED),    # L = 6
     ((1, 2, 4096, 64, 4, 5, 1, "bf16"), None),                     # p^(L-1) = 256: built
@@ -151,7 +152,7 @@ def test_entry_points_reject_bad_pointers_before_launching():
     assert b"aligned" in L.lh_last_error()
     assert L.lh_backward(ref, good, None, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
     assert L.lh_topk(ref, good, good, good, good, 16, None) == lh.LH_ERR_WORKSPACE
-    assert L.lh_attn_fwd(2, 100, 128, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_UNSUPPORTED
+    assert L.lh_attn_fwd(2, 100, 96, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_UNSUPPORTED
     assert L.lh_attn_fwd(0, 100, 64, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
     assert L.lh_attn_bwd_ws_bytes(2, 100, 64, lh.LH_BF16) >= 2 * 100 * 4
     assert L.lh_attn_bwd(2, 100, 64, lh.LH_BF16, good, good, good, good, good, good, None, good,

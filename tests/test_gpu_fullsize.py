@@ -1,13 +1,14 @@
 """Parity at the full benchmark sizes (98K and 512K tokens, 16 heads, bf16).
 
 The layer runs on the GPU exactly as the benchmark runs it (lh_forward /
-lh_backward on the whole [1, 16, N, 64] problem).  The oracle then checks
+lh_backward on the whole [1, H, N, d] problem).  The oracle then checks
 sampled heads: pyramid levels, scores and the selection in full; the
 attention output at sampled tokens (through the oracle's attention rows of
 the slots that reach them); and dQ/dK/dV on a 4096-token prefix (oracle
 backward restricted to the slots that reach the prefix, with the full
 forward's LSE and D), for every workload: 98K with k = 1536 and k = 6144,
-512K, 98K with p = 2, and 98K with the descent selection.
+512K, 98K with p = 2, 98K with the descent selection, and 98K with d = 128
+(8 heads).
 """
 import numpy as np
 import pytest
@@ -44,7 +45,7 @@ def _attention_rows_with_bounds(Qg, Kg, Vg, rows):
 
 
 @pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048", "98k_p2_k1536",
-                                        "98k_descent_k1536"])
+                                        "98k_descent_k1536", "98k_d128_k1536"])
 def run(request):
     from long_context_hierarchical_b200 import lh
     w = WORKLOADS[request.param]
@@ -64,6 +65,7 @@ def run(request):
 @pytest.mark.parametrize("h", HEADS)
 def test_fullsize_selection_and_output(run, h):
     w, pl, ctx = run["w"], run["pl"], run["ctx"]
+    h = min(h, w.H - 1)  # the d = 128 workload has 8 heads
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     Qh, Kh, Vh = (np64(run[x][0, h]) for x in ("Q", "K", "V"))
     # scores and selection, in full
@@ -124,7 +126,7 @@ def test_fullsize_gradient_prefix(run):
     with the full forward's LSE and D; the pool backward then gives the
     prefix tokens' gradients."""
     w, ctx = run["w"], run["ctx"]
-    h = HEADS[1]
+    h = min(HEADS[1], w.H - 1)
     sz = oracle.sizes(w.N, w.p, w.L, w.k)
     Qh, Kh, Vh, dOh = (np64(run[x][0, h]) for x in ("Q", "K", "V", "dO"))
     _, sel_idx, slot_of = oracle.head_select(Qh, Kh, sz, w.select)

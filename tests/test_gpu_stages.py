@@ -17,7 +17,7 @@ from tests.helpers import (TOL, assert_close, assert_grad_close, assert_pyr_clos
 
 pytestmark = pytest.mark.gpu
 
-# name: (B, H, N, dtype, p, L, k)
+# name: (B, H, N, dtype, p, L, k[, d]); d is 64 unless given
 CASES = {
     "tiny_f32": (1, 2, 1024, "f32", 4, 3, 32),          # S = 320
     "8k_bf16": (1, 8, 8192, "bf16", 4, 4, 256),         # S = 3200
@@ -29,6 +29,11 @@ CASES = {
     "kmax": (1, 2, 64, "bf16", 2, 2, 32),               # every candidate: S = 96
     "f32_p2_L5": (1, 1, 256, "f32", 2, 5, 3),           # S = 40
     "p2_L4_odd": (1, 2, 200, "bf16", 2, 4, 7),          # N = 25 * 8, S = 67
+    # head dimension 128
+    "d128_f32": (1, 2, 512, "f32", 4, 3, 16, 128),      # S = 160
+    "d128_ragged": (2, 3, 200, "bf16", 2, 4, 7, 128),   # S = 67: partial tiles and chunks
+    "d128_4k": (1, 4, 4096, "bf16", 4, 3, 64, 128),     # S = 768: six key tiles
+    "d128_L1_dense": (1, 2, 384, "bf16", 4, 1, 0, 128), # S = 384: a half-empty tile pair
 }
 
 DT = {"f32": torch.float32, "bf16": torch.bfloat16}
@@ -37,13 +42,14 @@ DT = {"f32": torch.float32, "bf16": torch.bfloat16}
 @pytest.fixture(scope="module", params=list(CASES))
 def case(request):
     from long_context_hierarchical_b200 import lh
-    B, H, N, dtype, p, L, k = CASES[request.param]
-    Q, K, V, dO = make_inputs(B, H, N, 64, dtype, seed=0)
+    B, H, N, dtype, p, L, k, *rest = CASES[request.param]
+    d = rest[0] if rest else 64
+    Q, K, V, dO = make_inputs(B, H, N, d, dtype, seed=0)
     O, ctxs, sz, grads = oracle_layer(Q, K, V, dO, p, L, k, DT[dtype])
-    pl = lh.plan(B, H, N, 64, p, L, k, dtype)
+    pl = lh.plan(B, H, N, d, p, L, k, dtype)
     dev = torch.device("cuda")
     terms = grad_tolerance_terms(ctxs, grads, sz)
-    return dict(name=request.param, B=B, H=H, N=N, dt=DT[dtype], p=p, L=L, k=k, lh=lh, pl=pl,
+    return dict(name=request.param, B=B, H=H, N=N, d=d, dt=DT[dtype], p=p, L=L, k=k, lh=lh, pl=pl,
                 Q=Q.to(dev), K=K.to(dev), V=V.to(dev), dO=dO.to(dev), O=O, ctxs=ctxs, sz=sz,
                 grads=grads, terms=terms)
 
@@ -59,7 +65,7 @@ def _oracle_pyr(c, which):
         hs = []
         for ctx in row:
             lv = ctx["levels"][which]
-            hs.append(np.concatenate(lv[1:], axis=0) if len(lv) > 1 else np.zeros((1, 64)))
+            hs.append(np.concatenate(lv[1:], axis=0) if len(lv) > 1 else np.zeros((1, c["d"])))
         rows.append(np.stack(hs))
     return np.stack(rows)
 
