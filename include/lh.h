@@ -178,10 +178,13 @@ int64_t lh_attn_bwd_ws_bytes(int64_t BH, int64_t S, int32_t d, int32_t dtype);
 /* Gradients of lh_attn_fwd.  D: [BH, S] fp32 rowsum(dOg * Og), or NULL, in
  * which case it is computed into ws from Og and dOg.  Writes dQg, dKg, dVg
  * [BH, S, d].  ws: lh_attn_bwd_ws_bytes() bytes.
- * bf16 runs one fused kernel by default: dQg is summed over key tiles with
- * fp32 atomics, so its last bits may differ between runs (dKg and dVg are
+ * bf16 runs one fused kernel by default: each key tile's share of dQg is
+ * added into an fp32 accumulator in ws with TMA bulk reduce-adds, whose order
+ * varies, so the last bits of dQg may differ between runs (dKg and dVg are
  * bit-reproducible).  lh_set_deterministic(1) selects a two-kernel schedule
- * without atomics (about 1.5x the time), as does lh_attn_bwd_static. */
+ * without reductions (dK/dV, then dQ per query tile; bit-reproducible and
+ * slower: about 1.6x the fused time at S = 18432), as does
+ * lh_attn_bwd_static. */
 lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, const void* Og, const float* lse,
                       const void* dOg, const float* D, void* dQg, void* dKg, void* dVg,
@@ -198,8 +201,8 @@ lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const voi
  * process exits.  Same arguments and results as lh_attn_bwd with D = NULL.
  *  - BH * S above LH_ATTN_BWD_STATIC_MAX_ROWS returns LH_ERR_WORKSPACE and
  *    enqueues nothing.
- *  - The first call on a device looks up the array's device address (a host
- *    call, once per device); make that first call before any stream capture.
+ *  - Every call looks up the array's device address in the current context
+ *    (a host-side call that enqueues nothing).
  *  - All calls share the one array and it keeps the last call's contents:
  *    calls whose work overlaps on the GPU (other streams, other threads) race
  *    on it and must be serialised by the caller.
@@ -236,15 +239,19 @@ lh_status lh_scatter_bwd(const lh_plan* plan, const void* dO, const void* Og,
 lh_status lh_gather_bwd(const lh_plan* plan, const void* dQg, const void* dKg, const void* dVg,
                         const int32_t* slot_of, void* dQ, void* dK, void* dV, lh_stream_t stream);
 
-/* Whole forward: O = layer(Q, K, V).  ctx: plan->ctx_bytes (kept for
- * lh_backward), ws: plan->ws_bytes of scratch. */
+/* Whole forward: O = layer(Q, K, V).  ctx (kept for lh_backward) and ws
+ * (scratch) are caller-owned device buffers of ctx_bytes and ws_bytes bytes;
+ * fewer than plan->ctx_bytes or plan->ws_bytes returns LH_ERR_WORKSPACE and
+ * enqueues nothing. */
 lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const void* V, void* O,
-                     void* ctx, void* ws, lh_stream_t stream);
+                     void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, lh_stream_t stream);
 
 /* Whole backward from the ctx of the matching lh_forward: dQ, dK, dV
- * [B,H,N,d] from dO.  ws: plan->ws_bytes of scratch. */
-lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void* dQ, void* dK,
-                      void* dV, void* ws, lh_stream_t stream);
+ * [B,H,N,d] from dO.  ctx_bytes, ws_bytes: the buffers' sizes, checked as in
+ * lh_forward. */
+lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, size_t ctx_bytes,
+                      void* dQ, void* dK, void* dV, void* ws, size_t ws_bytes,
+                      lh_stream_t stream);
 
 /* Device-side status word: LH_OK, or LH_ERR_TIMEOUT if a bounded wait inside
  * a kernel gave up since the last reset.  Synchronises the current device;

@@ -1,7 +1,6 @@
 // C-ABI entry points of the Lighthouse layer: validation, buffer layout and
 // the stage order of the whole forward and backward pass.
 #include <cuda_runtime.h>
-#include <nvtx3/nvToolsExt.h>
 #include <stdio.h>
 
 #include <string>
@@ -9,15 +8,6 @@
 #include "host.h"
 
 namespace lh {
-
-// NVTX range over one entry point or stage (a no-op unless a profiler is
-// attached), so a trace shows the stages by name around their launches.
-struct Range {
-  explicit Range(const char* name) { nvtxRangePushA(name); }
-  ~Range() { nvtxRangePop(); }
-  Range(const Range&) = delete;
-  Range& operator=(const Range&) = delete;
-};
 
 // Device status word (LH_OK or LH_ERR_TIMEOUT); kernels with bounded waits
 // receive its address from device_status_ptr().
@@ -77,6 +67,16 @@ int64_t attn_bwd_ws_bytes(int64_t BH, int64_t S, int d, int dtype);
 }  // namespace lh
 
 using namespace lh;
+
+lh_status lh::check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
+  if (BH < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "BH and S must be >= 1");
+  if (S >= (int64_t(1) << 31)) return fail(LH_ERR_INVALID_ARG, "S must stay below 2^31");
+  if (dtype != LH_F32 && dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
+  if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "only d in {64, 128} is built");
+  if (dtype == LH_BF16 && BH > ((int64_t(1) << 31) - 1) / S)
+    return fail(LH_ERR_UNSUPPORTED, "bf16 attention needs BH * S < 2^31 (TMA row coordinates)");
+  return LH_OK;
+}
 
 extern "C" {
 
@@ -278,15 +278,6 @@ lh_status lh_gather(const lh_plan* plan, const void* Q, const void* K, const voi
   return ok();
 }
 
-static lh_status check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype) {
-  if (BH < 1 || S < 1) return fail(LH_ERR_INVALID_ARG, "BH and S must be >= 1");
-  if (S >= (int64_t(1) << 31)) return fail(LH_ERR_INVALID_ARG, "S must stay below 2^31");
-  if (dtype != LH_F32 && dtype != LH_BF16) return fail(LH_ERR_UNSUPPORTED, "dtype must be LH_F32 or LH_BF16");
-  if (d != 64 && d != 128) return fail(LH_ERR_UNSUPPORTED, "only d in {64, 128} is built");
-  if (dtype == LH_BF16 && BH > ((int64_t(1) << 31) - 1) / S)
-    return fail(LH_ERR_UNSUPPORTED, "bf16 attention needs BH * S < 2^31 (TMA row coordinates)");
-  return LH_OK;
-}
 
 lh_status lh_attn_fwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, void* Og, float* lse, lh_stream_t stream) {
@@ -357,11 +348,15 @@ lh_status lh_gather_bwd(const lh_plan* plan, const void* dQg, const void* dKg, c
 }
 
 lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const void* V, void* O,
-                     void* ctx, void* ws, lh_stream_t stream) {
+                     void* ctx, size_t ctx_bytes, void* ws, size_t ws_bytes, lh_stream_t stream) {
   Range range("lh_forward");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(Q); LH_CHECK_PTR(K); LH_CHECK_PTR(V); LH_CHECK_PTR(O);
   LH_CHECK_PTR(ctx); LH_CHECK_PTR(ws);
+  if ((int64_t)ctx_bytes < plan->ctx_bytes)
+    return fail(LH_ERR_WORKSPACE, "lh_forward: ctx_bytes is below plan->ctx_bytes");
+  if ((int64_t)ws_bytes < plan->ws_bytes)
+    return fail(LH_ERR_WORKSPACE, "lh_forward: ws_bytes is below plan->ws_bytes");
   cudaStream_t st = as_cuda(stream);
   char* c = static_cast<char*>(ctx);
   char* w = static_cast<char*>(ws);
@@ -405,12 +400,16 @@ lh_status lh_forward(const lh_plan* plan, const void* Q, const void* K, const vo
   return ok();
 }
 
-lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, void* dQ, void* dK,
-                      void* dV, void* ws, lh_stream_t stream) {
+lh_status lh_backward(const lh_plan* plan, const void* dO, const void* ctx, size_t ctx_bytes,
+                      void* dQ, void* dK, void* dV, void* ws, size_t ws_bytes, lh_stream_t stream) {
   Range range("lh_backward");
   LH_TRY(check_plan(plan));
   LH_CHECK_PTR(dO); LH_CHECK_PTR(ctx); LH_CHECK_PTR(dQ); LH_CHECK_PTR(dK); LH_CHECK_PTR(dV);
   LH_CHECK_PTR(ws);
+  if ((int64_t)ctx_bytes < plan->ctx_bytes)
+    return fail(LH_ERR_WORKSPACE, "lh_backward: ctx_bytes is below plan->ctx_bytes");
+  if ((int64_t)ws_bytes < plan->ws_bytes)
+    return fail(LH_ERR_WORKSPACE, "lh_backward: ws_bytes is below plan->ws_bytes");
   cudaStream_t st = as_cuda(stream);
   const char* c = static_cast<const char*>(ctx);
   char* w = static_cast<char*>(ws);

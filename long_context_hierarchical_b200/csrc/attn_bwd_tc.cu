@@ -712,8 +712,10 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
       !make_tile_map(&kC, K, rows, C) || !make_tile_map(&vC, V, rows, C))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The opt-in to more than 48 KB of dynamic shared memory belongs to the
+  // function in the current device's context, so it is applied on every
+  // launch (a host-side call): right for any device, thread or context.
+  {
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<C, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, KV<C>::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -723,7 +725,6 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
     e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              QQ<C>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float sl2 = 0.125f * kLog2e;

@@ -626,8 +626,10 @@ cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
       !make_tile_map_d(&kC_, K, rows, kC, kD128) || !make_tile_map_d(&vC, V, rows, kC, kD128))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The opt-in to more than 48 KB of dynamic shared memory belongs to the
+  // function in the current device's context, so it is applied on every
+  // launch (a host-side call): right for any device, thread or context.
+  {
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc128_kernel<false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, KV::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -637,7 +639,6 @@ cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
     e = cudaFuncSetAttribute(attn_bwd_dq_tc128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              QQ::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float scale = (float)0.08838834764831845;  // 1/sqrt(128)

@@ -385,12 +385,13 @@ cudaError_t launch_attn_fwd_tc(int64_t BH, int64_t S, const void* Q, const void*
       !make_tile_map(&mv, V, BH * S, kRows))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The opt-in to more than 48 KB of dynamic shared memory belongs to the
+  // function in the current device's context, so it is applied on every
+  // launch (a host-side call): right for any device, thread or context.
+  {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int npairs = (int)((S + 2 * kRows - 1) / (2 * kRows));
   const float sl2 = 0.125f * 1.4426950408889634f;

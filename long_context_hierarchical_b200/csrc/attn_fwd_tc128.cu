@@ -314,12 +314,13 @@ cudaError_t launch_attn_fwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
       !make_tile_map_d(&mv, V, BH * S, kRows, kD128))
     return cudaErrorInvalidValue;
   unsigned int* status = device_status_ptr();
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The opt-in to more than 48 KB of dynamic shared memory belongs to the
+  // function in the current device's context, so it is applied on every
+  // launch (a host-side call): right for any device, thread or context.
+  {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc128_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int npairs = (int)((S + 2 * kRows - 1) / (2 * kRows));
   // 1/sqrt(128) * log2(e), rounded once

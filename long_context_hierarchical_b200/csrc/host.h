@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <string>
@@ -11,6 +12,15 @@
 
 namespace lh {
 
+// NVTX range over one entry point or stage (a no-op unless a profiler is
+// attached), so a trace shows the stages by name around their launches.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
+
 // Thread-local reason for the last non-OK status.
 lh_status fail(lh_status s, const std::string& why);
 lh_status ok();
@@ -18,6 +28,8 @@ lh_status ok();
 lh_status cuda_status(cudaError_t e, const char* where);
 
 Geo make_geo(const lh_plan& p);
+// Argument checks shared by the attention entry points (sizes, dtype, d).
+lh_status check_attn(int64_t BH, int64_t S, int32_t d, int32_t dtype);
 
 // Calls f.template operator()<T, D>() for the plan's storage type and head
 // dimension (d in {64, 128}, validated by lh_plan_init).

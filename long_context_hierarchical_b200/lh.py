@@ -84,8 +84,8 @@ def _load():
         "lh_scatter": (PLAN, P, P, P, P),
         "lh_scatter_bwd": (PLAN, P, P, P, P, P, P),
         "lh_gather_bwd": (PLAN, P, P, P, P, P, P, P, P),
-        "lh_forward": (PLAN, P, P, P, P, P, P, P),
-        "lh_backward": (PLAN, P, P, P, P, P, P, P),
+        "lh_forward": (PLAN, P, P, P, P, P, SZ, P, SZ, P),
+        "lh_backward": (PLAN, P, P, SZ, P, P, P, P, SZ, P),
         "lh_device_status": (ctypes.c_int,),
         "lh_selftest_wait_timeout": (P,),
         "lh_attn_bwd_static": (I64, I64, I32, I32, P, P, P, P, P, P, P, P, P, P),
@@ -415,7 +415,8 @@ def forward(pl: Plan, Q, K, V, O=None, ctx: Context | None = None, ws: Workspace
     _require(ctx.buf, "ctx", torch.uint8, pl.raw.ctx_bytes)
     _require(ws.buf, "ws", torch.uint8, pl.raw.ws_bytes)
     _check(LIB.lh_forward(pl.byref(), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(ctx.buf),
-                          _ptr(ws.buf), _stream(stream)), "lh_forward")
+                          ctx.buf.numel(), _ptr(ws.buf), ws.buf.numel(), _stream(stream)),
+           "lh_forward")
     return O, ctx
 
 
@@ -430,8 +431,9 @@ def backward(pl: Plan, dO, ctx: Context, dQ=None, dK=None, dV=None, ws: Workspac
     _require_tokens(pl, dQ=dQ, dK=dK, dV=dV)
     _require(ctx.buf, "ctx", torch.uint8, pl.raw.ctx_bytes)
     _require(ws.buf, "ws", torch.uint8, pl.raw.ws_bytes)
-    _check(LIB.lh_backward(pl.byref(), _ptr(dO), _ptr(ctx.buf), _ptr(dQ), _ptr(dK), _ptr(dV),
-                           _ptr(ws.buf), _stream(stream)), "lh_backward")
+    _check(LIB.lh_backward(pl.byref(), _ptr(dO), _ptr(ctx.buf), ctx.buf.numel(), _ptr(dQ),
+                           _ptr(dK), _ptr(dV), _ptr(ws.buf), ws.buf.numel(), _stream(stream)),
+           "lh_backward")
     return dQ, dK, dV
 
 

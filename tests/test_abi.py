@@ -147,10 +147,11 @@ def test_entry_points_reject_bad_pointers_before_launching():
     good = ctypes.c_void_p(1 << 20)       # aligned, never dereferenced here
     odd = ctypes.c_void_p((1 << 20) + 8)  # not 16-byte aligned
     L = lh.LIB
-    assert L.lh_forward(ref, None, good, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
-    assert L.lh_forward(ref, good, good, good, good, good, odd, None) == lh.LH_ERR_INVALID_ARG
+    cb, wb = p.raw.ctx_bytes, p.raw.ws_bytes
+    assert L.lh_forward(ref, None, good, good, good, good, cb, good, wb, None) == lh.LH_ERR_INVALID_ARG
+    assert L.lh_forward(ref, good, good, good, good, good, cb, odd, wb, None) == lh.LH_ERR_INVALID_ARG
     assert b"aligned" in L.lh_last_error()
-    assert L.lh_backward(ref, good, None, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
+    assert L.lh_backward(ref, good, None, cb, good, good, good, good, wb, None) == lh.LH_ERR_INVALID_ARG
     assert L.lh_topk(ref, good, good, good, good, 16, None) == lh.LH_ERR_WORKSPACE
     assert L.lh_attn_fwd(2, 100, 96, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_UNSUPPORTED
     assert L.lh_attn_fwd(0, 100, 64, lh.LH_BF16, good, good, good, good, good, None) == lh.LH_ERR_INVALID_ARG
@@ -161,6 +162,21 @@ def test_entry_points_reject_bad_pointers_before_launching():
     bad = lh.LhPlan.from_buffer_copy(p.raw)
     bad.S += 1
     assert L.lh_scatter(ctypes.byref(bad), good, good, good, None) == lh.LH_ERR_INVALID_ARG
+
+
+def test_whole_layer_calls_check_buffer_sizes_before_launching():
+    """lh_forward / lh_backward refuse a ctx or ws smaller than the plan's
+    (LH_ERR_WORKSPACE, nothing enqueued); the pointers are never touched."""
+    p = lh.plan(1, 2, 1024, 64, 4, 3, 8, "bf16")
+    ref, L = p.byref(), lh.LIB
+    good = ctypes.c_void_p(1 << 20)
+    cb, wb = p.raw.ctx_bytes, p.raw.ws_bytes
+    assert L.lh_forward(ref, good, good, good, good, good, cb - 1, good, wb, None) == lh.LH_ERR_WORKSPACE
+    assert b"ctx_bytes" in L.lh_last_error()
+    assert L.lh_forward(ref, good, good, good, good, good, cb, good, wb - 256, None) == lh.LH_ERR_WORKSPACE
+    assert b"ws_bytes" in L.lh_last_error()
+    assert L.lh_backward(ref, good, good, 0, good, good, good, good, wb, None) == lh.LH_ERR_WORKSPACE
+    assert L.lh_backward(ref, good, good, cb, good, good, good, good, 16, None) == lh.LH_ERR_WORKSPACE
 
 
 def test_status_strings():
