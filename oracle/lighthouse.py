@@ -37,6 +37,12 @@ Readings of points the pages leave open (each marked READING below):
      on to level 0.  Another reading of the budget (L-1)*p*k: p*k entries per
      finer level.  Needs k <= N/p^(L-1).  Coarse scores are the same
      max-pools as in R1; ties as in R3.
+  R9 (alternative selection, rule "regional") every region contributes: the
+     candidate score stream (level-major flat order) is cut into regions of
+     2048 entries (the pages' chunk size, the last one ragged); region c
+     keeps its floor(Ksel * |c| / M) best entries, and the Ksel - sum of
+     those go to the best of all entries not yet kept.  Ties as in R3.  The
+     budget and S stay those of R2.
 """
 from __future__ import annotations
 
@@ -228,6 +234,36 @@ def select_descent(cand, sz: Sizes):
         mask[sz.flat_off[l - 1] + children] = True
         current = children
         cur_scores = cand[sz.flat_off[l - 1] + children]
+    return mask
+
+
+REGION = 2048  # candidates per region of the regional rule (the pages' chunk size)
+
+
+def select_regional(cand, sz: Sizes, region: int = REGION):
+    """Boolean mask over all Ntot entries for the regional rule (READING R9).
+
+    The M candidate scores (levels 0..L-2, level-major) are cut into regions
+    of ``region`` consecutive entries; region c keeps its floor(Ksel * |c| /
+    M) best entries (ties to the lower flat index), so every part of the
+    sequence contributes; the rest of the budget goes to the best entries
+    not yet kept, over all regions.  Every coarsest-level entry is kept.
+    """
+    cand = np.asarray(cand, dtype=np.float64)
+    mask = np.zeros(sz.Ntot, dtype=bool)
+    mask[sz.flat_off[sz.L - 1]:] = True
+    if sz.Ksel == 0:
+        return mask
+    kept = np.zeros(sz.M, dtype=bool)
+    for a in range(0, sz.M, region):
+        b = min(sz.M, a + region)
+        quota = sz.Ksel * (b - a) // sz.M
+        best = np.argsort(-cand[a:b], kind="stable")[:quota]
+        kept[a + best] = True
+    rest = np.nonzero(~kept)[0]
+    extra = sz.Ksel - int(kept.sum())
+    kept[rest[np.argsort(-cand[rest], kind="stable")[:extra]]] = True
+    mask[: sz.M] = kept
     return mask
 
 
@@ -437,10 +473,12 @@ def gather_bwd(dXg, slot_of, sz: Sizes, mode: str):
 def head_select(Qh, Kh, sz: Sizes, rule: str = "joint"):
     """Scores, mask and order of one head (stages 2 and the ordering of 3).
 
-    rule: "joint" (READING R2) or "descent" (READING R8)."""
+    rule: "joint" (READING R2), "descent" (READING R8) or "regional"
+    (READING R9)."""
     s0 = level0_scores(Qh, Kh)
     cand = candidate_scores(s0, sz)
-    mask = select(cand, sz) if rule == "joint" else select_descent(cand, sz)
+    rules = {"joint": select, "descent": select_descent, "regional": select_regional}
+    mask = rules[rule](cand, sz)
     sel_idx, slot_of = order_selection(mask, sz)
     return cand, sel_idx, slot_of
 

@@ -321,6 +321,58 @@ def test_descent_needs_k_within_the_coarsest_level():
         lh.select_descent(np.zeros(sz.M), sz)
 
 
+def test_regional_hand_worked():
+    """The regional rule on the hand-worked scores, regions of 4 entries:
+    quotas 1, 1, 1 and one more entry from the best leftovers (a tie at 6
+    goes to the lower flat index 7)."""
+    g = GOLDEN["regional_select"]
+    sz = lh.sizes(g["N"], g["p"], g["L"], g["k"])
+    cand = np.array(g["cand"], float)
+    mask = lh.select_regional(cand, sz, region=g["region"])
+    kept = sorted(g["kept_by_region"] + g["kept_by_remainder"])
+    assert np.nonzero(mask[: sz.M])[0].tolist() == kept
+    assert lh.order_selection(mask, sz)[0].tolist() == g["sel_idx"]
+    # the joint rule keeps entry 11 instead of entry 1 on the same scores
+    assert not np.array_equal(lh.select(cand, sz), mask)
+
+
+@pytest.mark.parametrize("region", [1 << 20, 2048])
+def test_regional_is_joint_with_one_region(region):
+    """With a single region the quota is the whole budget: the joint rule."""
+    N, p, L, k = 1024, 4, 3, 16     # M = 1280 <= 2048
+    sz = lh.sizes(N, p, L, k)
+    cand = lh.candidate_scores(lh.level0_scores(rand_head(N, 8, 1), rand_head(N, 8, 2)), sz)
+    assert np.array_equal(lh.select_regional(cand, sz, region=region), lh.select(cand, sz))
+
+
+@pytest.mark.parametrize("N,p,L,k,region,distinct", [
+    (4096, 4, 3, 40, 512, None), (2400, 2, 3, 100, 2048, None), (4096, 4, 4, 30, 700, 3),
+    (2048, 2, 2, 1024, 300, None), (8192, 4, 4, 256, 2048, 1)])
+def test_regional_invariants(N, p, L, k, region, distinct):
+    """Exactly Ksel candidates; every region keeps at least its quota, and
+    its quota best entries (by score, then lower index) are among them; the
+    entries kept beyond the quotas beat every entry left out."""
+    sz = lh.sizes(N, p, L, k)
+    r = rng(N + region)
+    cand = r.standard_normal(sz.M)
+    if distinct:
+        cand = np.floor(r.random(sz.M) * distinct)
+    mask = lh.select_regional(cand, sz, region=region)
+    kept = mask[: sz.M]
+    assert kept.sum() == sz.Ksel and mask[sz.M:].all()
+    key = lambda f: (-cand[f], f)
+    extra_kept, left_out = [], []
+    for a in range(0, sz.M, region):
+        b = min(sz.M, a + region)
+        quota = sz.Ksel * (b - a) // sz.M
+        order = sorted(range(a, b), key=key)
+        assert kept[order[:quota]].all()
+        extra_kept += [f for f in order[quota:] if kept[f]]
+        left_out += [f for f in order[quota:] if not kept[f]]
+    if extra_kept and left_out:
+        assert max(key(f) for f in extra_kept) < min(key(f) for f in left_out)
+
+
 # --------------------------------------------------------------------------
 # stage 3: attention
 # --------------------------------------------------------------------------
