@@ -36,7 +36,8 @@
  * Readings of points the pages leave open (fixed by this library):
  *  - score of level-0 token t: ||Q_t||_2 + ||K_t||_2, computed in fp64 and
  *    rounded to fp32; coarser levels take the max over their span
- *    (gist.science 2.B: "coarser levels inherit scores ... via max-pooling").
+ *    (gist.science Technical Summary 2.B: a coarse entry takes the largest
+    score of the tokens it pools).
  *  - the budget: (L-1)*p*k entries chosen jointly from levels 0..L-2 by
  *    score, ties to the lower level-major flat index; the coarsest level is
  *    always kept in full (skill card, "阶段 2").
@@ -73,16 +74,23 @@ typedef enum { LH_F32 = 0, LH_BF16 = 1 } lh_dtype;
 /* Layer shape and hyperparameters.  p: pooling factor, L: pyramid levels
  * (level 0 = tokens), k: per-level budget unit, so (L-1)*p*k entries are
  * selected (skill card, "阶段 3").  The method needs N to be a multiple of
- * p^(L-1).  Built here: d = 64, p in {2, 4}, 1 <= L <= 5, p^(L-1) <= 256. */
+ * p^(L-1).  Built here: d in {64, 128}, p in {2, 4}, 1 <= L <= 5,
+ * p^(L-1) <= 256. */
 /* Selection rule for the (L-1)*p*k budget (lh_config.select):
  *  LH_SELECT_JOINT   one top-K of (L-1)*p*k over all candidate levels
  *                    0..L-2 (the default reading);
  *  LH_SELECT_DESCENT hierarchical descent: from the coarsest level down, the
  *                    k best entries of a level keep their p children one
- *                    level down (p*k per finer level); needs k <= n[L-1].
- * Both keep every coarsest-level entry and break ties to the lower
+ *                    level down (p*k per finer level); needs k <= n[L-1];
+ *  LH_SELECT_REGIONAL every region contributes (skill card "Kernel Design",
+ *                    chunked top-K): the M candidates, level-major, in
+ *                    regions of LH_REGION consecutive entries (the last one
+ *                    shorter); region c keeps its floor(Ksel*|c|/M) best and
+ *                    the remaining budget goes to the best entries left.
+ * All keep every coarsest-level entry and break ties to the lower
  * level-major flat index (skill card "阶段 2", "阶段 3"). */
-typedef enum { LH_SELECT_JOINT = 0, LH_SELECT_DESCENT = 1 } lh_select;
+typedef enum { LH_SELECT_JOINT = 0, LH_SELECT_DESCENT = 1, LH_SELECT_REGIONAL = 2 } lh_select;
+#define LH_REGION 2048
 
 typedef struct {
   int32_t B, H, N, d, p, L, k;
@@ -148,7 +156,8 @@ lh_status lh_pyramid_score(const lh_plan* plan, const void* Q, const void* K, co
  * plan's rule -- LH_SELECT_JOINT: the Ksel largest by (score desc, flat index
  * asc); LH_SELECT_DESCENT: the p children of the k best entries of each
  * level, from the coarsest down, a coarsest entry scoring the max of its p
- * children -- adds every level-(L-1) entry, and orders them by (span end,
+ * children; LH_SELECT_REGIONAL: each region's quota of its best entries,
+ * then the best of the rest -- adds every level-(L-1) entry, and orders them by (span end,
  * level).  sel_idx: [B,H,S] int32 flat indices in gathered order.  slot_of:
  * [B,H,Ntot] int32, the slot of each pyramid entry or -1.  ws:
  * plan->topk_ws_bytes of scratch (contents on entry are ignored). */
@@ -183,7 +192,7 @@ int64_t lh_attn_bwd_ws_bytes(int64_t BH, int64_t S, int32_t d, int32_t dtype);
  * varies, so the last bits of dQg may differ between runs (dKg and dVg are
  * bit-reproducible).  lh_set_deterministic(1) selects a two-kernel schedule
  * without reductions (dK/dV, then dQ per query tile; bit-reproducible and
- * slower: about 1.6x the fused time at S = 18432), as does
+ * slower: 1.5-1.6x the fused time at BH * S = 16 * 18432), as does
  * lh_attn_bwd_static. */
 lh_status lh_attn_bwd(int64_t BH, int64_t S, int32_t d, int32_t dtype, const void* Qg,
                       const void* Kg, const void* Vg, const void* Og, const float* lse,
@@ -219,7 +228,7 @@ lh_status lh_attn_bwd_static(int64_t BH, int64_t S, int32_t d, int32_t dtype, co
                              const void* Kg, const void* Vg, const void* Og, const float* lse,
                              const void* dOg, void* dQg, void* dKg, void* dVg, lh_stream_t stream);
 
-/* Stage 4 (skill card "阶段 4"; gist.science 2.C "deterministic scatter").
+/* Stage 4 (skill card "阶段 4"; gist.science 2.C: a deterministic scatter).
  * O[t] = sum over levels l (ascending) of Og[slot_of(l, floor((t+1)/p^l) - 1)]
  * where that index is >= 0 and selected; fp32 sum rounded once; 0 where no
  * entry reaches t.  O: [B,H,N,d].  No atomics. */

@@ -140,8 +140,9 @@ lh_status lh_plan_init(const lh_config* cfg, lh_plan* out) {
   p.Ksel = (int64_t)(c.L - 1) * c.p * c.k;
   if (p.Ksel > p.M) return fail(LH_ERR_INVALID_ARG, "(L-1)*p*k exceeds the candidate count");
   p.S = p.n[c.L - 1] + p.Ksel;
-  if (c.select != LH_SELECT_JOINT && c.select != LH_SELECT_DESCENT)
-    return fail(LH_ERR_INVALID_ARG, "select must be LH_SELECT_JOINT or LH_SELECT_DESCENT");
+  if (c.select != LH_SELECT_JOINT && c.select != LH_SELECT_DESCENT && c.select != LH_SELECT_REGIONAL)
+    return fail(LH_ERR_INVALID_ARG,
+                "select must be LH_SELECT_JOINT, LH_SELECT_DESCENT or LH_SELECT_REGIONAL");
   if (c.select == LH_SELECT_DESCENT && c.L >= 2 && c.k > p.n[c.L - 1])
     return fail(LH_ERR_INVALID_ARG, "descent selection needs k <= N / p^(L-1)");
   if (p.S >= (int64_t(1) << 31) || p.Ntot >= (int64_t(1) << 31))

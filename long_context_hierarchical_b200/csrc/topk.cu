@@ -16,7 +16,7 @@
 // two 12-bit histogram passes over the score bits, a compaction of the few
 // candidates left in the threshold bucket, and an 8-bit radix select on those.
 //
-// Order (stage 3 "密集子序列注意力"; gist.science 2.C "topologically sorted"):
+// Order (stage 3 "密集子序列注意力"; gist.science 2.C asks for a topological order):
 // selected entries are laid out by (last token of the span, level), which is
 // a walk over tokens t with, at each t, the levels l whose spans end at t
 // ((t + 1) % p^l == 0).  A count per token block, a scan of the block counts
@@ -30,6 +30,14 @@
 // candidates) and continues with those children.  A coarsest entry's score
 // is the maximum of its p children's, the same max-pool as the candidates'.
 // The ordering kernels then read the mask instead of a threshold.
+//
+// Regional rule (lh_select LH_SELECT_REGIONAL, the pages' chunked top-K with
+// every region contributing): one block per region of LH_REGION candidates
+// holds the region's keys in shared memory, finds the key of rank quota =
+// floor(Ksel * |region| / M) by the same radix select and marks the entries
+// at or above it; with R = Ksel - (sum of quotas) > 0 it also writes its R
+// best entries below that line to a list, and one block per (batch, head)
+// then keeps the R best keys of all regions' lists.
 //
 // Grid-wide phases are separate launches, and the reduction that closes a
 // phase runs in the last block to finish (an atomic ticket); no block ever
@@ -60,11 +68,22 @@ struct HeadState {
 static_assert(sizeof(HeadState) == 64, "HeadState is 64 bytes");
 
 constexpr int kDescThreads = 1024;
+constexpr int kRegThreads = 512;
 
 struct Layout {
   int64_t hist1, hist2, state, blockcnt, list, mask, keys, zero_bytes, total;
-  int64_t cap;  // descent: keys per level list
+  int64_t cap;   // descent: keys per level list
+  int64_t nreg;  // regional: regions of LH_REGION candidates
+  int64_t rest;  // regional: budget left after the regions' quotas
 };
+
+// Regional rule: Ksel minus the sum over regions of floor(Ksel * |region| / M).
+int64_t regional_rest(const lh_plan& p) {
+  int64_t q = 0;
+  for (int64_t a = 0; a < p.M; a += LH_REGION)
+    q += p.Ksel * (std::min<int64_t>(p.M, a + LH_REGION) - a) / p.M;
+  return p.Ksel - q;
+}
 
 int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
@@ -80,12 +99,18 @@ Layout layout(const lh_plan& p) {
   o = align256(o);
   l.blockcnt = o; o = align256(o + BH * nblk * 4);
   l.list = o; o = align256(o + BH * p.M * 8);
-  l.cap = 0;
+  l.cap = l.nreg = l.rest = 0;
   l.mask = l.keys = o;
   if (p.c.select == LH_SELECT_DESCENT && p.c.L >= 2) {
     l.cap = std::max<int64_t>(p.n[p.c.L - 1], (int64_t)p.c.p * p.c.k);
     l.mask = o; o = align256(o + BH * p.M);
     l.keys = o; o = align256(o + BH * 2 * l.cap * 8);
+  }
+  if (p.c.select == LH_SELECT_REGIONAL && p.M > 0) {
+    l.nreg = (p.M + LH_REGION - 1) / LH_REGION;
+    l.rest = regional_rest(p);
+    l.mask = o; o = align256(o + BH * p.M);
+    l.keys = o; o = align256(o + BH * l.nreg * l.rest * 8);
   }
   l.total = o;
   return l;
@@ -278,23 +303,25 @@ collect_kernel(Geo g, const float* __restrict__ scores, unsigned long long* list
 // --- hierarchical descent ----------------------------------------------------
 
 // The k-th largest of n unique keys (1 <= k <= n), by eight 8-bit radix passes
-// over the keys from the most significant digit.  Whole block.
+// over the keys from the most significant digit.  Whole block of NT threads.
+template <int NT>
 __device__ unsigned long long block_kth_largest(const unsigned long long* keys, int64_t n, uint32_t k,
                                                 uint32_t* h, uint32_t* warp_sums, uint32_t* s_digit,
                                                 uint32_t* s_need) {
+  static_assert(NT >= 256, "one thread per digit bin");
   unsigned long long prefix = 0, pmask = 0;
   uint32_t need = k;
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += kDescThreads) h[i] = 0;
+    for (int i = threadIdx.x; i < 256; i += NT) h[i] = 0;
     __syncthreads();
-    for (int64_t j = threadIdx.x; j < n; j += kDescThreads) {
+    for (int64_t j = threadIdx.x; j < n; j += NT) {
       const unsigned long long key = keys[j];
       if ((key & pmask) == prefix) atomicAdd(&h[(key >> shift) & 0xffu], 1u);
     }
     __syncthreads();
     const int t = threadIdx.x;
     const uint32_t v = t < 256 ? h[255 - t] : 0;  // descending digits
-    const uint32_t above = block_excl_scan<kDescThreads>(v, warp_sums, nullptr);
+    const uint32_t above = block_excl_scan<NT>(v, warp_sums, nullptr);
     if (t < 256 && above < need && need <= above + v) {
       *s_digit = 255 - t;
       *s_need = need - above;
@@ -331,7 +358,8 @@ descent_kernel(Geo g, const float* __restrict__ scores, uint8_t* __restrict__ ma
   }
   __syncthreads();
   for (int l = L - 1; l >= 1; --l) {
-    const unsigned long long kappa = block_kth_largest(cur, n, k, h, warp_sums, &s_digit, &s_need);
+    const unsigned long long kappa =
+        block_kth_largest<kDescThreads>(cur, n, k, h, warp_sums, &s_digit, &s_need);
     // keep the p children of every entry at or above kappa (exactly k of them)
     uint32_t base = 0;
     for (int64_t j0 = 0; j0 < n; j0 += kDescThreads) {
@@ -356,6 +384,74 @@ descent_kernel(Geo g, const float* __restrict__ scores, uint8_t* __restrict__ ma
     cur = nxt;
     nxt = t;
     n = (int64_t)p * k;
+  }
+}
+
+// --- regional rule -----------------------------------------------------------
+
+// One block per (region, head): the region's quota of best entries into the
+// mask (every candidate byte of the region is written), and with rest > 0
+// the region's `rest` best entries below the quota line into its list slot
+// (zero keys pad a short list; every real key is larger).
+__global__ void __launch_bounds__(kRegThreads)
+regional_kernel(Geo g, const float* __restrict__ scores, uint8_t* __restrict__ mask,
+                unsigned long long* __restrict__ rest_list, int64_t rest) {
+  __shared__ unsigned long long keys[LH_REGION];
+  __shared__ uint32_t h[256];
+  __shared__ uint32_t warp_sums[kRegThreads / 32];
+  __shared__ uint32_t s_digit, s_need;
+  const int64_t bh = blockIdx.y;
+  const int64_t a = (int64_t)blockIdx.x * LH_REGION;
+  const int64_t b = min(g.M, a + (int64_t)LH_REGION);
+  const int n = (int)(b - a);
+  const float* s = scores + bh * g.M;
+  for (int i = threadIdx.x; i < n; i += kRegThreads) keys[i] = full_key(s[a + i], a + i);
+  __syncthreads();
+  const uint32_t quota = (uint32_t)(g.Ksel * (b - a) / g.M);
+  unsigned long long kappa = 0;
+  if (quota > 0) kappa = block_kth_largest<kRegThreads>(keys, n, quota, h, warp_sums, &s_digit, &s_need);
+  uint8_t* msk = mask + bh * g.M + a;
+  for (int i = threadIdx.x; i < n; i += kRegThreads) msk[i] = (quota > 0 && keys[i] >= kappa) ? 1 : 0;
+  if (rest <= 0) return;
+  unsigned long long* out = rest_list + (bh * gridDim.x + blockIdx.x) * rest;
+  const uint32_t extra = (uint32_t)(rest < (int64_t)n - quota ? rest : (int64_t)n - quota);
+  if (extra > 0) {
+    const unsigned long long kappa2 =
+        block_kth_largest<kRegThreads>(keys, n, quota + extra, h, warp_sums, &s_digit, &s_need);
+    uint32_t base = 0;
+    for (int i0 = 0; i0 < n; i0 += kRegThreads) {
+      const int i = i0 + threadIdx.x;
+      const unsigned long long key = i < n ? keys[i] : 0ull;
+      const bool left = i < n && key >= kappa2 && !(quota > 0 && key >= kappa);
+      uint32_t total;
+      const uint32_t pos = base + block_excl_scan<kRegThreads>(left ? 1u : 0u, warp_sums, &total);
+      if (left && pos < extra) out[pos] = key;
+      base += total;
+    }
+  }
+  for (int64_t i = extra + threadIdx.x; i < rest; i += kRegThreads) out[i] = 0ull;
+}
+
+// One block per (batch, head): the `rest` best keys of all regions' lists
+// join the mask.
+__global__ void __launch_bounds__(kDescThreads)
+regional_rest_kernel(Geo g, uint8_t* __restrict__ mask, const unsigned long long* __restrict__ rest_list,
+                     int64_t nreg, int64_t rest) {
+  __shared__ uint32_t h[256];
+  __shared__ uint32_t warp_sums[kDescThreads / 32];
+  __shared__ uint32_t s_digit, s_need;
+  const int64_t bh = blockIdx.x;
+  const int64_t n = nreg * rest;
+  const unsigned long long* lst = rest_list + bh * n;
+  const unsigned long long kth =
+      block_kth_largest<kDescThreads>(lst, n, (uint32_t)rest, h, warp_sums, &s_digit, &s_need);
+  uint8_t* msk = mask + bh * g.M;
+  for (int64_t i = threadIdx.x; i < n; i += kDescThreads) {
+    const unsigned long long key = lst[i];
+    if (key != 0ull && key >= kth) {
+      const int64_t f = 0xffffffffll - (int64_t)(key & 0xffffffffull);
+      if (f >= 0 && f < g.M) msk[f] = 1;
+    }
   }
 }
 
@@ -467,8 +563,16 @@ cudaError_t launch_topk(const lh_plan& plan, const float* scores, int32_t* sel_i
   cudaError_t e = cudaMemsetAsync(w, 0, lay.zero_bytes, st);
   if (e != cudaSuccess) return e;
   const bool descent = g.select == LH_SELECT_DESCENT && g.Ksel > 0;
-  uint8_t* mask = descent ? reinterpret_cast<uint8_t*>(w + lay.mask) : nullptr;
-  if (descent) {
+  const bool regional = g.select == LH_SELECT_REGIONAL && g.Ksel > 0;
+  uint8_t* mask = (descent || regional) ? reinterpret_cast<uint8_t*>(w + lay.mask) : nullptr;
+  if (regional) {
+    // every candidate's mask byte is written by its region's block
+    unsigned long long* rl = reinterpret_cast<unsigned long long*>(w + lay.keys);
+    regional_kernel<<<dim3((unsigned)lay.nreg, (unsigned)g.BH), kRegThreads, 0, st>>>(g, scores, mask, rl,
+                                                                                     lay.rest);
+    if (lay.rest > 0)
+      regional_rest_kernel<<<(unsigned)g.BH, kDescThreads, 0, st>>>(g, mask, rl, lay.nreg, lay.rest);
+  } else if (descent) {
     e = cudaMemsetAsync(mask, 0, (size_t)(g.BH * g.M), st);
     if (e != cudaSuccess) return e;
     descent_kernel<<<(unsigned)g.BH, kDescThreads, 0, st>>>(

@@ -33,7 +33,7 @@ EXPORTS = (
 )
 
 
-SELECT = {"joint": 0, "descent": 1}
+SELECT = {"joint": 0, "descent": 1, "regional": 2}
 
 
 class LhConfig(ctypes.Structure):
@@ -210,8 +210,9 @@ class Plan:
 
 def plan(B: int, H: int, N: int, d: int = 64, p: int = 4, L: int = 3, k: int = 0,
          dtype: str = "bf16", select: str = "joint") -> Plan:
-    """select: "joint" (one top-K over all candidate levels) or "descent"
-    (hierarchical descent from the coarsest level)."""
+    """select: "joint" (one top-K over all candidate levels), "descent"
+    (hierarchical descent from the coarsest level) or "regional" (every
+    2048-candidate region keeps its share of the budget)."""
     cfg = LhConfig(B, H, N, d, p, L, k, DTYPES[dtype], SELECT[select])
     raw = LhPlan()
     _check(LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(raw)), "lh_plan_init")

@@ -35,7 +35,7 @@ class Workload:
     L: int
     k: int
     backward: bool  # the configuration the pages quote includes the backward pass
-    select: str = "joint"  # selection rule: "joint" or "descent"
+    select: str = "joint"  # selection rule: "joint", "descent" or "regional"
 
 
 # The workloads the layer is exercised and measured on.
@@ -50,6 +50,9 @@ WORKLOADS = {
     # the same budget chosen by hierarchical descent (k best per level, their children kept)
     "98k_descent_k1536": Workload("98k_descent_k1536", 1, 16, 98304, 64, "bf16", 4, 3, 1536, True,
                                   "descent"),
+    # the same budget with every 2048-candidate region keeping its share
+    "98k_regional_k1536": Workload("98k_regional_k1536", 1, 16, 98304, 64, "bf16", 4, 3, 1536, True,
+                                   "regional"),
     # head dimension 128 at the same bytes per token (8 heads x 128 channels)
     "98k_d128_k1536": Workload("98k_d128_k1536", 1, 8, 98304, 128, "bf16", 4, 3, 1536, True),
 }

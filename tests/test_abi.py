@@ -75,6 +75,17 @@ def test_plan_validation(args, status):
     assert e.value.status == status
 
 
+def test_plan_regional_selection_option():
+    """The regional rule keeps the same S and adds a candidate mask and the
+    regions' leftover lists to the top-K scratch; an unknown rule is refused."""
+    joint = lh.plan(1, 2, 8192, 64, 4, 4, 256, "bf16")
+    reg = lh.plan(1, 2, 8192, 64, 4, 4, 256, "bf16", select="regional")
+    assert reg.S == joint.S
+    assert reg.raw.topk_ws_bytes >= joint.raw.topk_ws_bytes + 2 * reg.M
+    cfg = lh.LhConfig(1, 2, 1024, 64, 4, 3, 8, lh.LH_BF16, 3)
+    assert lh.LIB.lh_plan_init(ctypes.byref(cfg), ctypes.byref(lh.LhPlan())) == lh.LH_ERR_INVALID_ARG
+
+
 def test_plan_descent_selection_option():
     """The descent rule keeps the same S, adds its scratch to the top-K
     workspace, and needs k <= N / p^(L-1)."""

@@ -45,7 +45,7 @@ def _attention_rows_with_bounds(Qg, Kg, Vg, rows):
 
 
 @pytest.fixture(scope="module", params=["98k_k1536", "98k_k6144", "512k_k2048", "98k_p2_k1536",
-                                        "98k_descent_k1536", "98k_d128_k1536"])
+                                        "98k_descent_k1536", "98k_regional_k1536", "98k_d128_k1536"])
 def run(request):
     from long_context_hierarchical_b200 import lh
     w = WORKLOADS[request.param]
@@ -114,7 +114,7 @@ def test_fullsize_selection_and_output(run, h):
                 exp_O[a] += Og[j]
                 term[a] += Tg[j]
                 spread[a] += Rg[j]
-    assert_grad_close(np64(run["O"][0, h])[tokens], _bf16(exp_O), Bound(term, spread, spread),
+    assert_grad_close(np64(run["O"][0, h])[tokens], _bf16(exp_O), Bound(term, spread, spread, spread),
                       torch.bfloat16, f"{w.name}:O sampled (head {h})")
 
 

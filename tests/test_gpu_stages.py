@@ -158,6 +158,58 @@ def test_descent_selection_on_seeded_scores(case):
     lh.device_status()
 
 
+# (B, H, N, p, L, k, distinct score levels or None): M spans several
+# 2048-candidate regions, a region straddling a level boundary, a ragged
+# last region, and a budget of every candidate
+REGIONAL_CASES = {
+    "p4_L3_3reg": (1, 3, 4096, 4, 3, 40, None),          # M = 5120: 2048, 2048, 1024
+    "p2_L3_straddle": (1, 2, 2400, 2, 3, 100, None),     # M = 3600: level 0 ends at 2400
+    "p4_L4_ties": (1, 2, 8192, 4, 4, 256, 3),            # M = 10752, three score values
+    "all_equal": (1, 1, 8192, 4, 4, 100, 1),
+    "everything": (1, 2, 4096, 2, 2, 2048, None),        # Ksel = M = 4096
+    "one_region": (1, 2, 1024, 4, 3, 16, None),          # M = 1280: the joint rule
+}
+
+
+@pytest.mark.parametrize("case", list(REGIONAL_CASES))
+def test_regional_selection_on_seeded_scores(case):
+    """Regional selection (LH_SELECT_REGIONAL) against the oracle's rule, bit
+    for bit, including ties everywhere and the budget of every candidate."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k, distinct = REGIONAL_CASES[case]
+    sz = oracle.sizes(N, p, L, k)
+    scores = make_scores(B, H, sz.M, seed=11, distinct=distinct)
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16", select="regional")
+    sel, inv = lh.topk(pl, scores.cuda())
+    for h in range(H):
+        mask = oracle.select_regional(scores[0, h].double().numpy(), sz)
+        es, ei = oracle.order_selection(mask, sz)
+        assert np.array_equal(sel[0, h].cpu().numpy(), es)
+        assert np.array_equal(inv[0, h].cpu().numpy(), ei)
+    lh.device_status()
+
+
+def test_regional_whole_layer():
+    """The whole layer with regional selection: selection bit-exact, output
+    and gradients within the attention tolerances."""
+    from long_context_hierarchical_b200 import lh
+    B, H, N, p, L, k = 1, 2, 4096, 4, 3, 48
+    Q, K, V, dO = make_inputs(B, H, N, 64, "bf16", seed=6)
+    O_e, ctxs, sz, grads = oracle_layer(Q, K, V, dO, p, L, k, torch.bfloat16, rule="regional")
+    terms = grad_tolerance_terms(ctxs, grads, sz)
+    pl = lh.plan(B, H, N, 64, p, L, k, "bf16", select="regional")
+    dev = [x.cuda() for x in (Q, K, V, dO)]
+    O, ctx = lh.forward(pl, *dev[:3])
+    g = lh.backward(pl, dev[3], ctx)
+    torch.cuda.synchronize()
+    assert np.array_equal(ctx.sel_idx.cpu().numpy(), stack(ctxs, "sel_idx"))
+    assert np.array_equal(ctx.slot_of.cpu().numpy(), stack(ctxs, "slot_of"))
+    assert_grad_close(np64(O), O_e, terms["O"], torch.bfloat16, "regional:O")
+    for got, i, key in ((g[0], 0, "dQ"), (g[1], 1, "dK"), (g[2], 2, "dV")):
+        assert_grad_close(np64(got), grads[i], terms[key], torch.bfloat16, f"regional:{key}")
+    lh.device_status()
+
+
 def test_descent_whole_layer():
     """The whole layer with descent selection: selection bit-exact, output
     and gradients within the attention tolerances."""
