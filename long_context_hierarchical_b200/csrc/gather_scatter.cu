@@ -104,6 +104,11 @@ template <int D>
 constexpr int kChunks = D / 8 / kLanesPerRow;  // 8-element chunks per lane
 constexpr int kRowsPerBlock4 = kThreads / kLanesPerRow;
 
+// Row loads of the token-centric kernels are issued for every level before
+// any of them is used: a level whose entry is not selected reads row 0 of
+// the head instead (valid memory, cached) and its value is dropped by a
+// select, so the sum and its order are those of a branch per level while
+// all L loads are in flight together.
 template <typename T, int D, int LOGP, int L>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
@@ -116,29 +121,31 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
   const T* og = Og + bh * g.S * D + c * 8;
   const int S = (int)g.S;
   int32_t slot[L];
+  bool hit[L];
 #pragma unroll
   for (int l = 0; l < L; ++l) {
     const int i = ((t + 1) >> (LOGP * l)) - 1;
-    slot[l] = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
+    const int32_t sl = i >= 0 ? __ldg(inv + (int)g.flat_off[l] + i) : -1;
+    hit[l] = (unsigned)sl < (unsigned)S;
+    slot[l] = hit[l] ? sl : 0;
   }
+  float x[L][kChunks<D>][8];
+#pragma unroll
+  for (int l = 0; l < L; ++l)
+#pragma unroll
+    for (int k = 0; k < kChunks<D>; ++k)
+      Vec8<T>::load(og + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
   float a[kChunks<D>][8];
 #pragma unroll
   for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
-  for (int l = 0; l < L; ++l) {  // ascending level
-    if ((unsigned)slot[l] < (unsigned)S) {
-      const T* src = og + (int64_t)slot[l] * D;
+  for (int l = 0; l < L; ++l)  // ascending level
 #pragma unroll
-      for (int k = 0; k < kChunks<D>; ++k) {
-        float x[8];
-        Vec8<T>::load(src + 8 * kLanesPerRow * k, x);
+    for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a[k][e] += x[e];
-      }
-    }
-  }
+      for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? a[k][e] + x[l][k][e] : a[k][e];
   T* dst = O + (bh * g.N + t) * D + c * 8;
 #pragma unroll
   for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
@@ -227,13 +234,24 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   const int64_t base = bh * g.S * D + c * 8;
   const int S = (int)g.S;
   int32_t slot[L];
+  bool hit[L];
 #pragma unroll
-  for (int l = 0; l < L; ++l) slot[l] = __ldg(inv + (int)g.flat_off[l] + (t >> (LOGP * l)));
+  for (int l = 0; l < L; ++l) {
+    const int32_t sl = __ldg(inv + (int)g.flat_off[l] + (t >> (LOGP * l)));
+    hit[l] = (unsigned)sl < (unsigned)S;
+    slot[l] = hit[l] ? sl : 0;
+  }
   const int64_t out = (bh * g.N + t) * D + c * 8;
   const T* src[3] = {dQg, dKg, dVg};
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
+    float x[L][kChunks<D>][8];
+#pragma unroll
+    for (int l = 0; l < L; ++l)
+#pragma unroll
+      for (int k = 0; k < kChunks<D>; ++k)
+        Vec8<T>::load(src[w] + base + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
     float a[kChunks<D>][8];
 #pragma unroll
     for (int k = 0; k < kChunks<D>; ++k)
@@ -241,17 +259,11 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
       for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
 #pragma unroll
     for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
-      if ((unsigned)slot[l] < (unsigned)S) {
-        const T* p = src[w] + base + (int64_t)slot[l] * D;
-        const float wgt = 1.f / (float)(1 << (LOGP * l));
+      const float wgt = 1.f / (float)(1 << (LOGP * l));
 #pragma unroll
-        for (int k = 0; k < kChunks<D>; ++k) {
-          float x[8];
-          Vec8<T>::load(p + 8 * kLanesPerRow * k, x);
+      for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a[k][e] = fmaf(x[e], wgt, a[k][e]);
-        }
-      }
+        for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? fmaf(x[l][k][e], wgt, a[k][e]) : a[k][e];
     }
 #pragma unroll
     for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst[w] + out + 8 * kLanesPerRow * k, a[k]);
