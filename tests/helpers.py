@@ -24,6 +24,10 @@ OPERAND_STEP = {torch.bfloat16: 2.0 ** -8, torch.float32: 2.0 ** -24}
 # spread over that interval, so its standard deviation is the bound over
 # sqrt(3): 2^-8 / sqrt(3) relative for a bf16 operand.
 SPREAD = {torch.bfloat16: 2.0 ** -8 / np.sqrt(3.0), torch.float32: 2.0 ** -24 / np.sqrt(3.0)}
+# fp32 error of forming a term before it is rounded (the dot products dP and
+# D accumulate in fp32, the exponent and the folded lse and D carry a few fp32
+# steps), relative to the sum of the magnitudes that enter it: 16 fp32 steps.
+FORM = 2.0 ** -20
 ROW_REL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
 HEAD_REL = {torch.bfloat16: 1e-2, torch.float32: 1e-5}
 RSS_SIGMAS = 4.0
@@ -39,11 +43,14 @@ class Bound(NamedTuple):
     l1:    sum over the terms of |term| (worst case: every rounding adds up);
     rss:   square root of the sum of squared rounded terms (the spread of
            independent roundings of the terms), given the oracle's Og;
-    rss_d: the same where the GPU formed its own Og, which shifts D.
+    rss_d: the same where the GPU formed its own Og, which shifts D;
+    rss_f: square root of the sum of squared magnitudes that enter each term
+           before its rounding (the spread of its fp32 formation errors).
     """
     l1: np.ndarray
     rss: np.ndarray
     rss_d: np.ndarray
+    rss_f: np.ndarray
 
 
 def np64(t):
@@ -93,8 +100,9 @@ def assert_pyr_close(got, exp, dtype, what, abs_mean=None, span=None):
 def _term_block(Qg, Kg, Vg, Og, lse, dOg, r0, r1, c1):
     """For query rows r0..r1-1 against keys < c1: P, the worst-case term
     factor P (|dP| + A) and the rounded operand dS = P (dP - D), where
-    A_i = sum_c |dOg_ic Og_ic|, D_i = sum_c dOg_ic Og_ic, and the root-sum-square
-    A2_i = (sum_c (dOg_ic Og_ic)^2)^(1/2)."""
+    A_i = sum_c |dOg_ic Og_ic|, D_i = sum_c dOg_ic Og_ic, the root-sum-square
+    A2_i = (sum_c (dOg_ic Og_ic)^2)^(1/2), and the magnitudes that enter dS
+    in fp32, F_ij = P_ij (sum_c |dOg_ic| |Vg_jc| + A_i)."""
     scale = 1.0 / np.sqrt(Qg.shape[1])
     s = (Qg[r0:r1] @ Kg[:c1].T) * scale
     rows = np.arange(r0, r1)[:, None]
@@ -104,7 +112,8 @@ def _term_block(Qg, Kg, Vg, Og, lse, dOg, r0, r1, c1):
     A = np.sum(np.abs(dOg[r0:r1] * Og[r0:r1]), axis=1)
     A2 = np.sqrt(np.sum((dOg[r0:r1] * Og[r0:r1]) ** 2, axis=1))
     D = np.sum(dOg[r0:r1] * Og[r0:r1], axis=1)
-    return P, P * (np.abs(dP) + A[:, None]), P * (dP - D[:, None]), A2
+    F = P * (np.abs(dOg[r0:r1]) @ np.abs(Vg[:c1]).T + A[:, None])
+    return P, P * (np.abs(dP) + A[:, None]), P * (dP - D[:, None]), A2, F
 
 
 def grad_term_bounds(Qg, Kg, Vg, Og, lse, dOg):
@@ -126,29 +135,39 @@ def grad_term_bounds(Qg, Kg, Vg, Og, lse, dOg):
     the root of the sum of the squared rounded terms: |dS_ij Kg_j| s,
     |dS_ij Qg_i| s, |P_ij dOg_i|, |P_ij Vg_j|.  Where the GPU forms its own
     Og (a whole layer) some of its elements round to the neighbouring bf16
-    value, which shifts D_i by a spread of about A2_i rounding steps and
-    moves every term of row i alike: one more term A2_i s |sum_j P_ij Kg_j|
-    for dQg_i, and P_ij A2_i |Qg_i| s per term of dKg_j.  Returns a dict of
-    ``Bound`` for dQg, dKg, dVg and Og.
+    value, one step (2^-7) away, which shifts D_i by a spread of about
+    2 A2_i rounding spreads and moves every term of row i alike: one more
+    term 2 A2_i s |sum_j P_ij Kg_j| for dQg_i, and 2 P_ij A2_i |Qg_i| s per
+    term of dKg_j.
+
+    rss_f: dS_ij is formed in fp32 from dP_ij and D_i, whose own sums cancel,
+    so its formation error scales with F_ij (``_term_block``): terms
+    F_ij |Kg_j| s and F_ij |Qg_i| s; for dVg and Og (P formed by the
+    exponential alone) the rss terms.  Returns a dict of ``Bound`` for dQg,
+    dKg, dVg and Og.
     """
     S, d = Qg.shape
     scale = 1.0 / np.sqrt(d)
     aK, aQ, aG, aV = np.abs(Kg), np.abs(Qg), np.abs(dOg), np.abs(Vg)
-    acc = {k: [np.zeros((S, d)) for _ in range(3)] for k in ("dQg", "dKg", "dVg", "Og")}
+    acc = {k: [np.zeros((S, d)) for _ in range(4)] for k in ("dQg", "dKg", "dVg", "Og")}
     for r0 in range(0, S, 512):
         r1 = min(S, r0 + 512)
-        P, T, dS, A2 = _term_block(Qg, Kg, Vg, Og, lse, dOg, r0, r1, r1)
+        P, T, dS, A2, F = _term_block(Qg, Kg, Vg, Og, lse, dOg, r0, r1, r1)
         acc["dQg"][0][r0:r1] = (T @ aK[:r1]) * scale
         acc["dQg"][1][r0:r1] = ((dS * dS) @ Kg[:r1] ** 2) * scale ** 2
-        acc["dQg"][2][r0:r1] = ((A2[:, None] * (P @ Kg[:r1])) ** 2) * scale ** 2
+        acc["dQg"][2][r0:r1] = ((2 * A2[:, None] * (P @ Kg[:r1])) ** 2) * scale ** 2
+        acc["dQg"][3][r0:r1] = ((F * F) @ Kg[:r1] ** 2) * scale ** 2
         acc["Og"][0][r0:r1] = P @ aV[:r1]
         acc["Og"][1][r0:r1] = (P * P) @ Vg[:r1] ** 2
         acc["dKg"][0][:r1] += (T.T @ aQ[r0:r1]) * scale
         acc["dKg"][1][:r1] += ((dS * dS).T @ Qg[r0:r1] ** 2) * scale ** 2
-        acc["dKg"][2][:r1] += ((P * P).T @ (A2[:, None] * Qg[r0:r1]) ** 2) * scale ** 2
+        acc["dKg"][2][:r1] += ((P * P).T @ (2 * A2[:, None] * Qg[r0:r1]) ** 2) * scale ** 2
+        acc["dKg"][3][:r1] += ((F * F).T @ Qg[r0:r1] ** 2) * scale ** 2
         acc["dVg"][0][:r1] += P.T @ aG[r0:r1]
         acc["dVg"][1][:r1] += (P * P).T @ dOg[r0:r1] ** 2
-    return {k: Bound(v[0], np.sqrt(v[1]), np.sqrt(v[1] + v[2])) for k, v in acc.items()}
+    for k in ("dVg", "Og"):
+        acc[k][3] = acc[k][1]
+    return {k: Bound(v[0], np.sqrt(v[1]), np.sqrt(v[1] + v[2]), np.sqrt(v[3])) for k, v in acc.items()}
 
 
 def grad_term_bounds_rows(Qg, Kg, Vg, Og, lse, dOg, q_rows, k_cols):
@@ -159,14 +178,15 @@ def grad_term_bounds_rows(Qg, Kg, Vg, Og, lse, dOg, q_rows, k_cols):
     q_rows = np.asarray(q_rows, dtype=np.int64)
     k_cols = np.asarray(k_cols, dtype=np.int64)
     out = {}
-    qq = [np.zeros((q_rows.size, d)) for _ in range(3)]
+    qq = [np.zeros((q_rows.size, d)) for _ in range(4)]
     for a, r in enumerate(q_rows):
-        P, T, dS, A2 = _term_block(Qg, Kg, Vg, Og, lse, dOg, r, r + 1, r + 1)
+        P, T, dS, A2, F = _term_block(Qg, Kg, Vg, Og, lse, dOg, r, r + 1, r + 1)
         qq[0][a] = (T @ np.abs(Kg[: r + 1]))[0] * scale
         qq[1][a] = ((dS * dS) @ Kg[: r + 1] ** 2)[0] * scale ** 2
-        qq[2][a] = ((A2[:, None] * (P @ Kg[: r + 1])) ** 2)[0] * scale ** 2
-    out["dQg"] = Bound(qq[0], np.sqrt(qq[1]), np.sqrt(qq[1] + qq[2]))
-    kk = [np.zeros((k_cols.size, d)) for _ in range(5)]
+        qq[2][a] = ((2 * A2[:, None] * (P @ Kg[: r + 1])) ** 2)[0] * scale ** 2
+        qq[3][a] = ((F * F) @ Kg[: r + 1] ** 2)[0] * scale ** 2
+    out["dQg"] = Bound(qq[0], np.sqrt(qq[1]), np.sqrt(qq[1] + qq[2]), np.sqrt(qq[3]))
+    kk = [np.zeros((k_cols.size, d)) for _ in range(6)]
     for a, c in enumerate(k_cols):
         P = np.exp((Qg[c:] @ Kg[c]) * scale - lse[c:])
         A = np.sum(np.abs(dOg[c:] * Og[c:]), axis=1)
@@ -175,13 +195,15 @@ def grad_term_bounds_rows(Qg, Kg, Vg, Og, lse, dOg, q_rows, k_cols):
         dP = dOg[c:] @ Vg[c]
         T = P * (np.abs(dP) + A)
         dS = P * (dP - D)
+        F = P * (np.abs(dOg[c:]) @ np.abs(Vg[c]) + A)
         kk[0][a] = (T @ np.abs(Qg[c:])) * scale
         kk[1][a] = ((dS * dS) @ Qg[c:] ** 2) * scale ** 2
-        kk[4][a] = ((P * P * A2 * A2) @ Qg[c:] ** 2) * scale ** 2
+        kk[4][a] = ((P * P * 4 * A2 * A2) @ Qg[c:] ** 2) * scale ** 2
+        kk[5][a] = ((F * F) @ Qg[c:] ** 2) * scale ** 2
         kk[2][a] = P @ np.abs(dOg[c:])
         kk[3][a] = (P * P) @ dOg[c:] ** 2
-    out["dKg"] = Bound(kk[0], np.sqrt(kk[1]), np.sqrt(kk[1] + kk[4]))
-    out["dVg"] = Bound(kk[2], np.sqrt(kk[3]), np.sqrt(kk[3]))
+    out["dKg"] = Bound(kk[0], np.sqrt(kk[1]), np.sqrt(kk[1] + kk[4]), np.sqrt(kk[5]))
+    out["dVg"] = Bound(kk[2], np.sqrt(kk[3]), np.sqrt(kk[3]), np.sqrt(kk[3]))
     return out
 
 
@@ -192,20 +214,20 @@ def grad_tolerance_terms(ctxs, grads, sz):
     and a token's output at most L; both bounds add up over those rows
     (for the root-sum-square bound that is the triangle inequality)."""
     keys = ("dQg", "dKg", "dVg", "dQ", "dK", "dV", "Og", "O")
-    out = {k: ([], [], []) for k in keys}
+    out = {k: ([], [], [], []) for k in keys}
     for crow, grow in zip(ctxs, grads[3]):
-        r = {k: ([], [], []) for k in keys}
+        r = {k: ([], [], [], []) for k in keys}
         for ctx, g in zip(crow, grow):
             b = grad_term_bounds(ctx["Qg"], ctx["Kg"], ctx["Vg"], ctx["Og"], ctx["lse"], g["dOg"])
             for key in ("dQ", "dK", "dV"):
-                for i in range(3):
+                for i in range(4):
                     r[key + "g"][i].append(b[key + "g"][i])
                     r[key][i].append(oracle.gather_bwd(b[key + "g"][i], ctx["slot_of"], sz, "f64"))
-            for i in range(3):
+            for i in range(4):
                 r["Og"][i].append(b["Og"][i])
                 r["O"][i].append(oracle.scatter(b["Og"][i], ctx["slot_of"], sz, "f64"))
         for k in keys:
-            for i in range(3):
+            for i in range(4):
                 out[k][i].append(np.stack(r[k][i]))
     return {k: Bound(*(np.stack(x) for x in v)) for k, v in out.items()}
 
@@ -217,19 +239,22 @@ def cancelling_sum_errors(got, exp, terms, dtype, own_og=True):
       elem: |g - o| / (TOL max(1, |o|) + 2 step |terms|_1)  per element, with
             step = 2^-8 (bf16 operands; two roundings reach each term, so
             2 step = 2^-7) -- the worst case;
-      row:  ||g_r - o_r|| / (ROW_REL ||o_r|| + RSS_SIGMAS SPREAD ||rss_r||)
-            per row r over the channels: independent roundings of the terms
-            add up like a random walk, so an element's spread is SPREAD rss
-            and a row's the norm of those; ROW_REL covers the roundings of
-            the stored result (the gathered and the final gradient);
-      head: ||g - o|| / (HEAD_REL ||o|| + RSS_SIGMAS SPREAD ||rss||) per head.
+      row:  ||g_r - o_r|| / (ROW_REL ||o_r|| + RSS_SIGMAS ||sigma_r||) per
+            row r over the channels, where an element's spread sigma is
+            ((SPREAD rss)^2 + (FORM rss_f)^2)^(1/2): independent roundings of
+            the terms add up like a random walk; ROW_REL covers the
+            roundings of the stored result (the gathered and the final
+            gradient);
+      head: ||g - o|| / (HEAD_REL ||o|| + RSS_SIGMAS ||sigma||) per head.
     ``own_og``: the GPU formed Og itself (a whole layer), so D may shift
     (``Bound.rss_d``); False where the stage was fed the oracle's Og.
     """
     got = np.asarray(got, dtype=np.float64)
     exp = np.asarray(exp, dtype=np.float64)
     if isinstance(terms, Bound):
-        l1, rss = terms.l1, (terms.rss_d if own_og else terms.rss)
+        l1 = terms.l1
+        rss = np.sqrt((SPREAD[dtype] * (terms.rss_d if own_og else terms.rss)) ** 2
+                      + (FORM * terms.rss_f) ** 2)
     else:
         l1, rss = terms, np.zeros_like(exp)
     step = OPERAND_STEP[dtype]
@@ -238,11 +263,11 @@ def cancelling_sum_errors(got, exp, terms, dtype, own_og=True):
     elem = err / (base + 2 * step * l1)
     e_r = np.sqrt(np.sum(err ** 2, axis=-1))
     row = e_r / (ROW_REL[dtype] * np.sqrt(np.sum(exp ** 2, axis=-1))
-                 + RSS_SIGMAS * SPREAD[dtype] * np.sqrt(np.sum(rss ** 2, axis=-1)) + 1e-30)
+                 + RSS_SIGMAS * np.sqrt(np.sum(rss ** 2, axis=-1)) + 1e-30)
     hx = lambda a: np.sqrt(np.sum(a.reshape(-1, a.shape[-2] * a.shape[-1]) ** 2, axis=1)) \
         if a.ndim >= 2 else np.sqrt(np.sum(a ** 2))[None]
     e_h, o_h, s_h = hx(err), hx(exp), hx(rss)
-    head = e_h / (HEAD_REL[dtype] * o_h + RSS_SIGMAS * SPREAD[dtype] * s_h + 1e-30)
+    head = e_h / (HEAD_REL[dtype] * o_h + RSS_SIGMAS * s_h + 1e-30)
     nz = np.abs(exp) > 0
     ulp = err[nz] / bf16_ulp(exp[nz]) if nz.any() else np.zeros(1)
     return {

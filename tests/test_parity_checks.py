@@ -103,6 +103,6 @@ def test_bound_without_spread_terms_is_elementwise_only():
     exp = np.ones((2, 3, 4))
     st = cancelling_sum_errors(exp * (1 + 1e-3), exp, np.zeros_like(exp), BF16)
     assert st["elem_margin"] < 1 and st["row_margin"] < 1 and st["head_margin"] < 1
-    b = Bound(np.zeros_like(exp), np.zeros_like(exp), np.zeros_like(exp))
+    b = Bound(*(np.zeros_like(exp),) * 4)
     st = cancelling_sum_errors(exp * 1.03, exp, b, BF16)
     assert st["row_margin"] > 1 and st["head_margin"] > 1
