@@ -104,7 +104,8 @@ class ClockSampler:
 STAGES = ("pyramid_score", "topk", "gather", "attn_fwd", "scatter",
           "scatter_bwd", "attn_bwd", "gather_bwd")
 # kernels each stage launches (lh_topk also issues one cudaMemsetAsync)
-# kernels per stage (top-K: 5 for the joint rule, 3 for the descent rule)
+# kernels per stage (top-K: 5 for the joint rule, 3 for the descent rule, 4
+# for the regional rule)
 LAUNCHES = {"pyramid_score": 1, "topk": 5, "gather": 1, "attn_fwd": 1, "scatter": 1,
             "scatter_bwd": 1, "attn_bwd": 2, "gather_bwd": 1}
 
@@ -209,6 +210,19 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def cpu_sample_inputs(w, seed, head):
     """One (b, h) head of the workload's seeded inputs, as fp64 arrays."""
     Q, K, V, dO = make_workload_inputs(w, seed=seed, device="cpu")
@@ -238,6 +252,7 @@ def run_reference(args, w, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": blas_threads(), "kind": "oracle",
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model(),
                          "sample": f"one (b,h) head of {heads} per step, full forward+backward of "
                                    f"that head; time x {heads} heads"},
         "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -288,6 +303,29 @@ def timed_steps(layer, st, steps, backward=True):
     return total / steps, [x / steps for x in per_stage]
 
 
+def sdpa_backend(q, k, v):
+    """The backend torch's causal SDPA dispatches to for these tensors
+    (torch's own backend choice), with the kernel its profiler shows when
+    one can be captured."""
+    from torch.nn.attention import SDPBackend
+    names = {int(getattr(SDPBackend, n)): n.lower() for n in dir(SDPBackend) if n.isupper()}
+    try:
+        choice = names.get(int(torch._fused_sdp_choice(q, k, v, None, 0.0, True)), "unknown")
+    except Exception:
+        choice = "unknown"
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+            torch.cuda.synchronize()
+        kernels = [e.name for e in prof.events() if e.device_type.name == "CUDA"]
+        if kernels:
+            choice += f" ({max(kernels, key=len)[:80]})"
+    except Exception:
+        pass
+    return choice
+
+
 def dense_sdpa_ms(H, N, steps=3, backward=True, d=64):
     q = torch.randn(1, H, N, d, device="cuda", dtype=torch.bfloat16, requires_grad=backward)
     k = torch.randn_like(q, requires_grad=backward)
@@ -307,22 +345,96 @@ def dense_sdpa_ms(H, N, steps=3, backward=True, d=64):
         once()
     b.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps
+    backend = None if backward else sdpa_backend(q.detach(), k.detach(), v.detach())
+    return a.elapsed_time(b) / steps, backend
 
 
-def workload_extras(w, fwd_ms, fb_ms, dense_steps=3):
-    """Forward / forward+backward throughput and dense causal SDPA at the same N."""
+def dense_own_ms(lh, H, N, d, steps=1):
+    """The build's own causal attention kernels (lh_attn_fwd / lh_attn_bwd) on
+    the whole sequence, S = N: the second dense comparator."""
+    g = torch.Generator(device="cuda").manual_seed(1)
+    mk = lambda: torch.randn(H, N, d, device="cuda", dtype=torch.bfloat16, generator=g)
+    q, k, v, do = mk(), mk(), mk(), mk()
+    o, lse = lh.attn_fwd(q, k, v)
+    lh.attn_bwd(q, k, v, o, lse, do, None)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for _ in range(steps):
+        o, lse = lh.attn_fwd(q, k, v)
+    ev[1].record()
+    for _ in range(steps):
+        lh.attn_bwd(q, k, v, o, lse, do, None)
+    ev[2].record()
+    torch.cuda.synchronize()
+    f = ev[0].elapsed_time(ev[1]) / steps
+    b = ev[1].elapsed_time(ev[2]) / steps
+    del q, k, v, do, o, lse
+    torch.cuda.empty_cache()
+    return f, f + b
+
+
+def workload_extras(lh, w, fwd_ms, fb_ms, dense_steps=3):
+    """Forward / forward+backward throughput and the two dense causal
+    comparators at the same N: torch SDPA and the build's own kernels."""
     out = {"fwd_ms": fwd_ms, "fwd_bwd_ms": fb_ms,
            "fwd_mtok_s": w.B * w.N / (fwd_ms * 1e-3) / 1e6,
            "fwd_bwd_mtok_s": w.B * w.N / (fb_ms * 1e-3) / 1e6}
     try:
-        sd_f = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False, d=w.d)
-        sd_fb = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True, d=w.d)
-        out["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb,
+        sd_f, backend = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False, d=w.d)
+        sd_fb, _ = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True, d=w.d)
+        out["dense_sdpa_torch"] = {"fwd_ms": sd_f, "fwd_bwd_ms": sd_fb, "backend": backend,
                                    "speedup_fwd": sd_f / fwd_ms, "speedup_fwd_bwd": sd_fb / fb_ms}
     except Exception as e:  # comparator only
         out["dense_sdpa_torch"] = {"error": str(e)[:200]}
     torch.cuda.empty_cache()
+    try:
+        own_f, own_fb = dense_own_ms(lh, w.B * w.H, w.N, w.d)
+        out["dense_own_kernels"] = {"fwd_ms": own_f, "fwd_bwd_ms": own_fb,
+                                    "speedup_fwd": own_f / fwd_ms, "speedup_fwd_bwd": own_fb / fb_ms}
+    except Exception as e:  # comparator only
+        out["dense_own_kernels"] = {"error": str(e)[:200]}
+    torch.cuda.empty_cache()
+    return out
+
+
+def stage_rooflines(pl, w, per_stage, peaks):
+    """Per stage: time, algorithmic work, rate, and fraction of the measured
+    peak (HBM copy for memory-bound stages; bf16 burst and sustained for the
+    attention kernels)."""
+    work = stage_work(pl, w)
+    stages = {}
+    for name, t_ms in zip(STAGES, per_stage):
+        kind, amount = work[name]
+        if kind == "bytes":
+            gbs = amount / (t_ms * 1e-3) / 1e9
+            stages[name] = {"ms": t_ms, "bytes": amount, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]}
+        else:
+            tf = amount / (t_ms * 1e-3) / 1e12
+            stages[name] = {"ms": t_ms, "flops": amount, "TFLOP/s": tf,
+                            "frac_tensor": tf / peaks["bf16"],
+                            "frac_tensor_sustained": tf / peaks["bf16_sus"]}
+    return stages
+
+
+def measure_workload(lh, stp, name, steps=3, dense_steps=1):
+    """A further workload: its layer step stage by stage, forward only, and
+    the dense comparators at its N."""
+    w = WORKLOADS[name]
+    Q, K, V, dO = make_workload_inputs(w, seed=0, device="cuda")
+    layer = Layer(lh, w, Q, K, V, dO)
+    for _ in range(3):
+        layer.step(stp)
+    torch.cuda.synchronize()
+    fb, st = timed_steps(layer, stp, steps)
+    f, _ = timed_steps(layer, stp, steps, backward=False)
+    pl = layer.pl
+    del layer, Q, K, V, dO
+    torch.cuda.empty_cache()
+    out = workload_extras(lh, w, f, fb, dense_steps=dense_steps)
+    out["config"] = {k: getattr(w, k) for k in ("B", "H", "N", "d", "p", "L", "k", "select")}
+    out["S"] = pl.S
+    out["stages"] = stage_rooflines(pl, w, st, load_peaks())
     return out
 
 
@@ -376,17 +488,7 @@ def main():
     tokens = w.B * w.N * world
     value = throughput(w.B * w.N, world, ms)
     peaks = load_peaks()
-    work = stage_work(layer.pl, w)
-    stages = {}
-    for name, t_ms in zip(STAGES, per_stage):
-        kind, amount = work[name]
-        if kind == "bytes":
-            gbs = amount / (t_ms * 1e-3) / 1e9
-            stages[name] = {"ms": t_ms, "bytes": amount, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]}
-        else:
-            tf = amount / (t_ms * 1e-3) / 1e12
-            stages[name] = {"ms": t_ms, "flops": amount, "TFLOP/s": tf,
-                            "frac_tensor": tf / peaks["bf16_sus"]}
+    stages = stage_rooflines(layer.pl, w, per_stage, peaks)
     dom = max(STAGES, key=lambda s: stages[s]["ms"])
     d = stages[dom]
     traffic = None
@@ -394,9 +496,13 @@ def main():
     if os.path.exists(tpath):
         traffic = json.load(open(tpath)).get(f"lh_{dom}@{w.name}")
     if "flops" in d:
+        # the timed region is short (steps x ms_per_step) and runs at full
+        # clock, so the burst figure is the denominator; the sustained one
+        # (measured under the power cap) is reported beside it
         roof = {"kernel": f"lh_{dom}", "bound": "tensor", "achieved": d["TFLOP/s"],
-                "peak": peaks["bf16_sus"], "unit": "TFLOP/s", "frac": d["frac_tensor"],
-                "traffic": traffic, "peak_source": f"{peaks['src']} bf16 sustained"}
+                "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": d["frac_tensor"],
+                "traffic": traffic, "peak_source": f"{peaks['src']} bf16 burst",
+                "frac_of_sustained": d["frac_tensor_sustained"]}
     else:
         roof = {"kernel": f"lh_{dom}", "bound": "hbm", "achieved": d["GB/s"], "peak": peaks["hbm"],
                 "unit": "GB/s", "frac": d["frac_hbm"], "traffic": traffic,
@@ -431,27 +537,20 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         fwd_ms, _ = timed_steps(layer, stp, args.steps, backward=False)
-        extras[w.name] = workload_extras(w, fwd_ms, ms)
+        extras[w.name] = workload_extras(lh, w, fwd_ms, ms)
         del layer, Q, K, V, dO, hQ, hK, hV, hdO, hO, hdQ, hdK, hdV
         torch.cuda.empty_cache()
-        if w.name != "512k_k2048":
-            w5 = WORKLOADS["512k_k2048"]
-            Q5, K5, V5, dO5 = make_workload_inputs(w5, seed=0, device="cuda")
-            l5 = Layer(lh, w5, Q5, K5, V5, dO5)
-            for _ in range(2):
-                l5.step(stp)
-            torch.cuda.synchronize()
-            fb5, st5 = timed_steps(l5, stp, 3)
-            f5, _ = timed_steps(l5, stp, 3, backward=False)
-            extras[w5.name] = workload_extras(w5, f5, fb5, dense_steps=1)
-            extras[w5.name]["stages_ms"] = dict(zip(STAGES, st5))
-            del l5, Q5, K5, V5, dO5
-            torch.cuda.empty_cache()
+        # the other configurations of the pages' measurements, each once:
+        # 98K with k = 6144, 512K, head dimension 128, pooling p = 2
+        for name, dense_steps in (("98k_k6144", 1), ("512k_k2048", 1), ("98k_d128_k1536", 1),
+                                  ("98k_p2_k1536", 1)):
+            if name != w.name:
+                extras[name] = measure_workload(lh, stp, name, dense_steps=dense_steps)
         Qh, Kh, Vh, dOh = cpu_sample_inputs(w, 0, 0)
         secs = oracle_head_seconds(w, Qh, Kh, Vh, dOh)
         heads = w.B * w.H
         cpu = {"value": w.B * w.N / (secs * heads) / 1e6, "unit": "Mtok/s", "cores": blas_threads(),
-               "kind": "oracle",
+               "kind": "oracle", "nproc": os.cpu_count(), "cpu_model": cpu_model(),
                "sample": f"one (b,h) head of {heads}: full forward+backward of that head, "
                          f"{secs:.1f} s, scaled x {heads} heads"}
 
@@ -467,7 +566,8 @@ def main():
                     "ms_per_step": e2e_ms,
                     "schedule": "lh.HostPipeline: step i's kernels overlap the copy-in of "
                                 "step i+1 and the copy-out of step i-1"},
-            "gpu_launches": (sum(LAUNCHES.values()) - (2 if w.select == "descent" else 0)) * args.steps,
+            "gpu_launches": (sum(LAUNCHES.values())
+                             - {"joint": 0, "descent": 2, "regional": 1}[w.select]) * args.steps,
             "clocks": clk, "stages": stages, "extras": extras,
         }
         print(json.dumps(line), flush=True)
