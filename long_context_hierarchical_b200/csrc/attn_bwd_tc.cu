@@ -728,10 +728,11 @@ cudaError_t launch_attn_bwd_tc(int64_t BH, int64_t S, const void* Q, const void*
   }
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float sl2 = 0.125f * kLog2e;
-  // (problems, tiles): every problem's longest tile is launched before any
-  // shorter one, which keeps the tail of the grid short
-  const int ty = ntiles <= 65535 ? 1 : 0;
-  if (!ty && BH > 65535) return cudaErrorInvalidConfiguration;
+  // (tiles, problems): one problem's key tiles are launched together,
+  // longest first, so the operands and fp32 dQ accumulator of one or two
+  // problems at a time stay in L2 (faster than interleaving the problems)
+  const int ty = BH > 65535 ? 1 : 0;
+  if (ty && ntiles > 65535) return cudaErrorInvalidConfiguration;
   const dim3 grid = ty ? dim3((unsigned)BH, ntiles) : dim3(ntiles, (unsigned)BH);
   if (dq_acc != nullptr) {
     const int64_t n = BH * S * kD;

@@ -643,8 +643,11 @@ cudaError_t launch_attn_bwd_tc128(int64_t BH, int64_t S, const void* Q, const vo
   const int ntiles = (int)((S + kRows - 1) / kRows);
   const float scale = (float)0.08838834764831845;  // 1/sqrt(128)
   const float sl2 = (float)(0.08838834764831845 * 1.4426950408889634);
-  const int ty = ntiles <= 65535 ? 1 : 0;
-  if (!ty && BH > 65535) return cudaErrorInvalidConfiguration;
+  // (tiles, problems): one problem's key tiles are launched together,
+  // longest first, so the operands and fp32 dQ accumulator of one or two
+  // problems at a time stay in L2 (faster than interleaving the problems)
+  const int ty = BH > 65535 ? 1 : 0;
+  if (ty && ntiles > 65535) return cudaErrorInvalidConfiguration;
   const dim3 grid = ty ? dim3((unsigned)BH, ntiles) : dim3(ntiles, (unsigned)BH);
   if (dq_acc != nullptr) {
     const int64_t n = rows * kD128;
