@@ -376,10 +376,13 @@ def dense_own_ms(lh, H, N, d, steps=1):
 
 def workload_extras(lh, w, fwd_ms, fb_ms, dense_steps=3):
     """Forward / forward+backward throughput and the two dense causal
-    comparators at the same N: torch SDPA and the build's own kernels."""
+    comparators at the same N: torch SDPA and the build's own kernels
+    (dense_steps = 0: no comparators)."""
     out = {"fwd_ms": fwd_ms, "fwd_bwd_ms": fb_ms,
            "fwd_mtok_s": w.B * w.N / (fwd_ms * 1e-3) / 1e6,
            "fwd_bwd_mtok_s": w.B * w.N / (fb_ms * 1e-3) / 1e6}
+    if dense_steps <= 0:
+        return out
     try:
         sd_f, backend = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=False, d=w.d)
         sd_fb, _ = dense_sdpa_ms(w.H, w.N, steps=dense_steps, backward=True, d=w.d)
@@ -541,9 +544,12 @@ def main():
         del layer, Q, K, V, dO, hQ, hK, hV, hdO, hO, hdQ, hdK, hdV
         torch.cuda.empty_cache()
         # the other configurations of the pages' measurements, each once:
-        # 98K with k = 6144, 512K, head dimension 128, pooling p = 2
+        # 98K with k = 6144, 512K, head dimension 128, pooling p = 2; and the
+        # two other selection rules at 98K (their dense comparators are the
+        # default workload's)
         for name, dense_steps in (("98k_k6144", 1), ("512k_k2048", 1), ("98k_d128_k1536", 1),
-                                  ("98k_p2_k1536", 1)):
+                                  ("98k_p2_k1536", 1), ("98k_regional_k1536", 0),
+                                  ("98k_descent_k1536", 0)):
             if name != w.name:
                 extras[name] = measure_workload(lh, stp, name, dense_steps=dense_steps)
         Qh, Kh, Vh, dOh = cpu_sample_inputs(w, 0, 0)

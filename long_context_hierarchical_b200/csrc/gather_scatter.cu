@@ -104,12 +104,15 @@ template <int D>
 constexpr int kChunks = D / 8 / kLanesPerRow;  // 8-element chunks per lane
 constexpr int kRowsPerBlock4 = kThreads / kLanesPerRow;
 
-// Row loads of the token-centric kernels are issued for every level before
-// any of them is used: a level whose entry is not selected reads row 0 of
-// the head instead (valid memory, cached) and its value is dropped by a
-// select, so the sum and its order are those of a branch per level while
-// all L loads are in flight together.
-template <typename T, int D, int LOGP, int L>
+// Two forms of the token-centric kernels, with the same sums in the same
+// order.  kAll: the row loads of every level are issued before any of them
+// is used, so all L are in flight together (a level whose entry is not
+// selected reads row 0 of the head instead, valid cached memory, and drops
+// the value with a select); this is faster where most tokens have several
+// selected levels (98K tokens, k = 1536: S/N = 0.19).  Otherwise a branch per
+// level loads only the selected rows, faster for sparse selections (512K,
+// k = 2048: S/N = 0.06).  The launch picks kAll for S/N >= 1/8.
+template <typename T, int D, int LOGP, int L, bool kAll>
 __global__ void __launch_bounds__(kThreads)
 scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot_of,
                T* __restrict__ O) {
@@ -129,23 +132,38 @@ scatter_kernel(Geo g, const T* __restrict__ Og, const int32_t* __restrict__ slot
     hit[l] = (unsigned)sl < (unsigned)S;
     slot[l] = hit[l] ? sl : 0;
   }
-  float x[L][kChunks<D>][8];
-#pragma unroll
-  for (int l = 0; l < L; ++l)
-#pragma unroll
-    for (int k = 0; k < kChunks<D>; ++k)
-      Vec8<T>::load(og + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
   float a[kChunks<D>][8];
 #pragma unroll
   for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
     for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
+  if constexpr (kAll) {
+    float x[L][kChunks<D>][8];
 #pragma unroll
-  for (int l = 0; l < L; ++l)  // ascending level
+    for (int l = 0; l < L; ++l)
 #pragma unroll
-    for (int k = 0; k < kChunks<D>; ++k)
+      for (int k = 0; k < kChunks<D>; ++k)
+        Vec8<T>::load(og + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? a[k][e] + x[l][k][e] : a[k][e];
+    for (int l = 0; l < L; ++l)  // ascending level
+#pragma unroll
+      for (int k = 0; k < kChunks<D>; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? a[k][e] + x[l][k][e] : a[k][e];
+  } else {
+#pragma unroll
+    for (int l = 0; l < L; ++l) {  // ascending level
+      if (hit[l]) {
+#pragma unroll
+        for (int k = 0; k < kChunks<D>; ++k) {
+          float x[8];
+          Vec8<T>::load(og + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[k][e] += x[e];
+        }
+      }
+    }
+  }
   T* dst = O + (bh * g.N + t) * D + c * 8;
 #pragma unroll
   for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst + 8 * kLanesPerRow * k, a[k]);
@@ -221,7 +239,7 @@ scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
   if (c == 0) Drow[r] = dsum;
 }
 
-template <typename T, int D, int LOGP, int L>
+template <typename T, int D, int LOGP, int L, bool kAll>
 __global__ void __launch_bounds__(kThreads)
 gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
                   const T* __restrict__ dVg, const int32_t* __restrict__ slot_of,
@@ -246,24 +264,40 @@ gather_bwd_kernel(Geo g, const T* __restrict__ dQg, const T* __restrict__ dKg,
   T* dst[3] = {dQ, dK, dV};
 #pragma unroll
   for (int w = 0; w < 3; ++w) {
-    float x[L][kChunks<D>][8];
-#pragma unroll
-    for (int l = 0; l < L; ++l)
-#pragma unroll
-      for (int k = 0; k < kChunks<D>; ++k)
-        Vec8<T>::load(src[w] + base + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
     float a[kChunks<D>][8];
 #pragma unroll
     for (int k = 0; k < kChunks<D>; ++k)
 #pragma unroll
       for (int e = 0; e < 8; ++e) a[k][e] = 0.f;
+    if constexpr (kAll) {
+      float x[L][kChunks<D>][8];
 #pragma unroll
-    for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
-      const float wgt = 1.f / (float)(1 << (LOGP * l));
+      for (int l = 0; l < L; ++l)
 #pragma unroll
-      for (int k = 0; k < kChunks<D>; ++k)
+        for (int k = 0; k < kChunks<D>; ++k)
+          Vec8<T>::load(src[w] + base + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x[l][k]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? fmaf(x[l][k][e], wgt, a[k][e]) : a[k][e];
+      for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
+        const float wgt = 1.f / (float)(1 << (LOGP * l));
+#pragma unroll
+        for (int k = 0; k < kChunks<D>; ++k)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[k][e] = hit[l] ? fmaf(x[l][k][e], wgt, a[k][e]) : a[k][e];
+      }
+    } else {
+#pragma unroll
+      for (int l = 0; l < L; ++l) {  // ascending level; 1/p^l is a power of two: exact
+        if (hit[l]) {
+          const float wgt = 1.f / (float)(1 << (LOGP * l));
+#pragma unroll
+          for (int k = 0; k < kChunks<D>; ++k) {
+            float x[8];
+            Vec8<T>::load(src[w] + base + (int64_t)slot[l] * D + 8 * kLanesPerRow * k, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[k][e] = fmaf(x[e], wgt, a[k][e]);
+          }
+        }
+      }
     }
 #pragma unroll
     for (int k = 0; k < kChunks<D>; ++k) store_stream<T>(dst[w] + out + 8 * kLanesPerRow * k, a[k]);
@@ -310,11 +344,18 @@ void with_levels(const Geo& g, F&& f) {
   }
 }
 
+// The all-levels form for selections of at least one slot per 8 tokens.
+bool dense_selection(const Geo& g) { return 8 * g.S >= g.N; }
+
 template <typename T, int D>
 void scatter_t(const Geo& g, const void* Og, const int32_t* slot_of, void* O, cudaStream_t st) {
   const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
+  const bool all = dense_selection(g);
   with_levels(g, [&]<int LOGP, int L>() {
-    scatter_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+    if (all)
+      scatter_kernel<T, D, LOGP, L, true><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
+    else
+      scatter_kernel<T, D, LOGP, L, false><<<grid, kThreads, 0, st>>>(g, (const T*)Og, slot_of, (T*)O);
   });
 }
 
@@ -348,9 +389,14 @@ template <typename T, int D>
 void gather_bwd_t(const Geo& g, const void* dQg, const void* dKg, const void* dVg,
                   const int32_t* slot_of, void* dQ, void* dK, void* dV, cudaStream_t st) {
   const dim3 grid(blocks_for4(g.N), (unsigned)g.BH);
+  const bool all = dense_selection(g);
   with_levels(g, [&]<int LOGP, int L>() {
-    gather_bwd_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(
-        g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
+    if (all)
+      gather_bwd_kernel<T, D, LOGP, L, true><<<grid, kThreads, 0, st>>>(
+          g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
+    else
+      gather_bwd_kernel<T, D, LOGP, L, false><<<grid, kThreads, 0, st>>>(
+          g, (const T*)dQg, (const T*)dKg, (const T*)dVg, slot_of, (T*)dQ, (T*)dK, (T*)dV);
   });
 }
 
