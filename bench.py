@@ -420,13 +420,13 @@ def stage_rooflines(pl, w, per_stage, peaks):
     return stages
 
 
-def measure_workload(lh, stp, name, steps=3, dense_steps=1):
+def measure_workload(lh, stp, name, steps=10, dense_steps=1):
     """A further workload: its layer step stage by stage, forward only, and
     the dense comparators at its N."""
     w = WORKLOADS[name]
     Q, K, V, dO = make_workload_inputs(w, seed=0, device="cuda")
     layer = Layer(lh, w, Q, K, V, dO)
-    for _ in range(3):
+    for _ in range(5):
         layer.step(stp)
     torch.cuda.synchronize()
     fb, st = timed_steps(layer, stp, steps)
