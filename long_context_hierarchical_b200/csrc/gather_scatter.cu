@@ -174,15 +174,60 @@ template <int D>
 constexpr int kBwdChunks = D / 8 / kBwdLanes;
 constexpr int kRowsPerBlockB = kThreads / kBwdLanes;
 
-template <typename T, int D, int LOGP, int L>
+// Position, within its block, of the slot row that slot group `grp` handles
+// when the block's rows are taken level by level: the rows of one level share
+// one range length, so a warp's row sums mostly share one trip count.  Rows
+// past S sort last.  Which group takes which row varies from run to run; each
+// row's result does not.
+template <int L>
+__device__ __forceinline__ int slot_by_level(const Geo& g, const int32_t* __restrict__ sel_row,
+                                             int first, int grp, int c) {
+  __shared__ int s_level[kRowsPerBlockB];
+  __shared__ int s_start[L + 1];
+  __shared__ int s_order[kRowsPerBlockB];
+  if (threadIdx.x <= L) s_start[threadIdx.x] = 0;
+  __syncthreads();
+  if (c == 0) {
+    int lv = L;
+    if (first + grp < (int)g.S) {
+      int f = sel_row[first + grp];
+      if (f < 0 || f >= (int)g.Ntot) f = (int)g.Ntot - 1;  // unreachable for a valid selection
+      lv = 0;
+#pragma unroll
+      for (int q = 1; q < L; ++q)
+        if (f >= (int)g.flat_off[q]) lv = q;
+    }
+    s_level[grp] = lv;
+    atomicAdd(&s_start[lv], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {  // counts -> exclusive prefix
+    int run = 0;
+    for (int q = 0; q <= L; ++q) {
+      const int n = s_start[q];
+      s_start[q] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (c == 0) s_order[atomicAdd(&s_start[s_level[grp]], 1)] = grp;
+  __syncthreads();
+  return s_order[grp];
+}
+
+template <typename T, int D, int LOGP, int L, bool kByLevel>
 __global__ void __launch_bounds__(kThreads)
 scatter_bwd_kernel(Geo g, const T* __restrict__ dO, const T* __restrict__ Og,
                    const int32_t* __restrict__ sel_idx, T* __restrict__ dOg, float* __restrict__ Drow) {
-  const int j = blockIdx.x * kRowsPerBlockB + (int)(threadIdx.x / kBwdLanes);
+  const int64_t bh = blockIdx.y;
+  const int first = blockIdx.x * kRowsPerBlockB;
+  const int grp = (int)(threadIdx.x / kBwdLanes);
   const int c = threadIdx.x % kBwdLanes;
+  int jj = grp;
+  if constexpr (kByLevel) jj = slot_by_level<L>(g, sel_idx + bh * g.S, first, grp, c);
+  const int j = first + jj;
   const int S = (int)g.S, N = (int)g.N;
   const bool live = j < S;
-  const int64_t bh = blockIdx.y;
   const int64_t r = bh * g.S + (live ? j : 0);
   int f = sel_idx[r];
   if (f < 0 || f >= (int)g.Ntot) f = (int)g.Ntot - 1;  // unreachable for a valid selection
@@ -370,9 +415,17 @@ template <typename T, int D>
 void scatter_bwd_t(const Geo& g, const void* dO, const void* Og, const int32_t* sel_idx, void* dOg,
                    float* Drow, cudaStream_t st) {
   const dim3 grid((unsigned)((g.S + kRowsPerBlockB - 1) / kRowsPerBlockB), (unsigned)g.BH);
+  // Sparse selections mix long coarse ranges with single tokens inside one
+  // block; taking the rows level by level pays there (0.273 vs 0.296 ms at
+  // 512K tokens, 4 heads) and not for dense ones (0.073 vs 0.071 ms at 98K).
+  const bool by_level = !dense_selection(g);
   with_levels(g, [&]<int LOGP, int L>() {
-    scatter_bwd_kernel<T, D, LOGP, L><<<grid, kThreads, 0, st>>>(g, (const T*)dO, (const T*)Og,
-                                                                 sel_idx, (T*)dOg, Drow);
+    if (by_level)
+      scatter_bwd_kernel<T, D, LOGP, L, true><<<grid, kThreads, 0, st>>>(
+          g, (const T*)dO, (const T*)Og, sel_idx, (T*)dOg, Drow);
+    else
+      scatter_bwd_kernel<T, D, LOGP, L, false><<<grid, kThreads, 0, st>>>(
+          g, (const T*)dO, (const T*)Og, sel_idx, (T*)dOg, Drow);
   });
 }
 
