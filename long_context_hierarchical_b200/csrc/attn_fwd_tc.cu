@@ -172,13 +172,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       auto step = [&](int x, int j, int n) -> bool {
         if (j + 1 < n) {
           const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
-          if (!mbar_wait(bars + kBarSF + 8 * x, j & 1, abort, status)) return false;
-          if (!mbar_wait(bars + kBarK + 8 * s1, u1 & 1, abort, status)) return false;
+          if (!mbar_wait2(bars + kBarSF + 8 * x, j & 1, bars + kBarK + 8 * s1, u1 & 1, abort, status))
+            return false;
           tc_fence_after();
           issue_S(x, j + 1);
         }
-        if (!mbar_wait(bars + kBarP + 8 * x, j & 1, abort, status)) return false;
-        if (!mbar_wait(bars + kBarV + 8 * (j % kStages), (j / kStages) & 1, abort, status)) return false;
+        if (!mbar_wait2(bars + kBarP + 8 * x, j & 1, bars + kBarV + 8 * (j % kStages), (j / kStages) & 1,
+                        abort, status))
+          return false;
         tc_fence_after();
         issue_PV(x, j);
         return true;

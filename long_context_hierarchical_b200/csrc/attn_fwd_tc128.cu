@@ -176,8 +176,9 @@ attn_fwd_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
       };
       // tile x at key tile j: P_x(j) V_j, then S_x(j+1) over the same columns
       auto step = [&](int x, int j, int n) -> bool {
-        if (!mbar_wait(bars + kBarP + 8 * x, j & 1, abort, status)) return false;
-        if (!mbar_wait(bars + kBarV + 8 * (j % kStages), (j / kStages) & 1, abort, status)) return false;
+        if (!mbar_wait2(bars + kBarP + 8 * x, j & 1, bars + kBarV + 8 * (j % kStages), (j / kStages) & 1,
+                        abort, status))
+          return false;
         tc_fence_after();
         issue_PV(x, j);
         if (j + 1 < n) {

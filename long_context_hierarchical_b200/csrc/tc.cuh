@@ -69,6 +69,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Two phases tested together, so that the latencies of the two tests overlap
+// when both are already complete (a single issuing thread waits on two
+// barriers before most of its MMAs: 3.5 % of the forward at 98K tokens);
+// otherwise each is waited for in turn, with mbar_wait's bound.
+__device__ __forceinline__ bool mbar_wait2(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1,
+                                           volatile int* abort, unsigned int* status) {
+  const bool d0 = mbar_try_wait(b0, p0);
+  const bool d1 = mbar_try_wait(b1, p1);
+  if (d0 && d1) return true;
+  return (d0 || mbar_wait(b0, p0, abort, status)) && (d1 || mbar_wait(b1, p1, abort, status));
+}
+
 // 2-D TMA tile load into this CTA's own shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
