@@ -292,12 +292,15 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
       for (int t = 0; ok && t < nq; ++t) {
         const int s = t % kStages;
         // S^T/dP^T of step t copied out: start step t+1's while step t computes
-        if (!(ok = mbar_wait(bars + L::kBarTF, t & 1, abort, status))) break;
-        tc_fence_after();
         if (t + 1 < nq) {
           const int s1 = (t + 1) % kStages, u1 = (t + 1) / kStages;
-          if (!(ok = mbar_wait(bars + L::kBarFull + 8 * s1, u1 & 1, abort, status))) break;
+          if (!(ok = mbar_wait2(bars + L::kBarTF, t & 1, bars + L::kBarFull + 8 * s1, u1 & 1, abort, status)))
+            break;
+          tc_fence_after();
           issue_sp(s1);
+        } else {
+          if (!(ok = mbar_wait(bars + L::kBarTF, t & 1, abort, status))) break;
+          tc_fence_after();
         }
         if constexpr (kFused) {
           if (t >= 2) {  // share t-2's reduce has read the boxes
@@ -353,8 +356,7 @@ attn_bwd_dkdv_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
     bool ok = true;
     for (int t = 0; t < nq; ++t) {
       const int s = t % kStages;
-      ok = mbar_wait(bars + L::kBarSP, t & 1, abort, status);
-      if (ok) ok = mbar_wait(bars + L::kBarFull + 8 * s, (t / kStages) & 1, abort, status);
+      ok = mbar_wait2(bars + L::kBarSP, t & 1, bars + L::kBarFull + 8 * s, (t / kStages) & 1, abort, status);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
       const int q0 = k0 + t * kC;
@@ -532,8 +534,8 @@ attn_bwd_dq_tc128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
         tc_fence_after();
         if (j + 1 < nk) {
           const int s1 = (j + 1) % kStages, u1 = (j + 1) / kStages;
-          if (!(ok = mbar_wait(bars + L::kBarK + 8 * s1, u1 & 1, abort, status))) break;
-          if (!(ok = mbar_wait(bars + L::kBarV + 8 * s1, u1 & 1, abort, status))) break;
+          if (!(ok = mbar_wait2(bars + L::kBarK + 8 * s1, u1 & 1, bars + L::kBarV + 8 * s1, u1 & 1, abort, status)))
+            break;
           gemm_rc(tmem, base + L::kOffQ, base + L::kOffK + s1 * kTileC);
           gemm_rc(tmem + kC, base + L::kOffG, base + L::kOffV + s1 * kTileC);
           mma_commit(bars + L::kBarSP);
