@@ -29,6 +29,9 @@ CASES = {
     "kmax": (1, 2, 64, "bf16", 2, 2, 32),               # every candidate: S = 96
     "f32_p2_L5": (1, 1, 256, "f32", 2, 5, 3),           # S = 40
     "p2_L4_odd": (1, 2, 200, "bf16", 2, 4, 7),          # N = 25 * 8, S = 67
+    # S = 1792 < N / 8: the token kernels' sparse forms (a branch per level;
+    # scatter backward rows taken level by level) over 28 slot blocks
+    "sparse_64k": (1, 2, 65536, "bf16", 4, 4, 64),
     # head dimension 128
     "d128_f32": (1, 2, 512, "f32", 4, 3, 16, 128),      # S = 160
     "d128_ragged": (2, 3, 200, "bf16", 2, 4, 7, 128),   # S = 67: partial tiles and chunks
